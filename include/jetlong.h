@@ -1,0 +1,157 @@
+/*
+ * jetlong.h -- C ABI of libjetlong.so: Jet-Long dynamic bifocal RoPE attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
+ * RoPE" (Tang, Wang, Gu, Han, Cai, 2026), as summarised on the web pages
+ * gist.science/es, gist.science/de and gist.science/ja (Methodology sections
+ * 1 and 2) and in the abstract on chatpaper.ai/fr.
+ *
+ * Notation.  L: length of a sequence (prefill) or of the cache including the
+ * current token (decode).  w_pretrained: pretraining window.  w0: local window.
+ * G = max(1, ceil(L / w_pretrained)); f(x) = floor(x / G).  A (query i, key j)
+ * pair with 0 <= i - j < w0 is LOCAL and scores <R(i)q, R(j)k>; any other
+ * causal pair is REMOTE and scores <R(f(i))q, R(f(j))k>.  R(p) is RoPE in the
+ * rotate-half pairing (c, c + d/2) with theta_c = rope_base^(-2c/d).
+ * Query head h reads KV head floor(h / (Hq / Hkv)).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them.  bf16 tensors are token-major and contiguous.
+ *    Every tensor pointer must be 16-byte aligned.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Nothing blocks the host except jl_sync_status.
+ *  - Arguments are validated before anything is launched.  A failed check
+ *    returns JL_ERR_INVALID (or JL_ERR_UNSUPPORTED for a valid but unbuilt
+ *    shape) and sets a thread-local message readable with jl_last_error().
+ *    A CUDA launch failure returns JL_ERR_CUDA.
+ *  - Kernels never trap.  Every wait inside a kernel is bounded; a wait that
+ *    runs out records JL_ERR_TIMEOUT in a device status word and the kernel
+ *    returns.  jl_sync_status() reports and clears that word.
+ *  - Only sm_100a is built.  There is no CPU fallback.
+ */
+#ifndef JETLONG_H
+#define JETLONG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* jl_stream_t;
+
+typedef enum {
+  JL_OK = 0,
+  JL_ERR_INVALID = 1,     /* bad argument; nothing was launched                */
+  JL_ERR_UNSUPPORTED = 2, /* valid request for a shape this build does not have */
+  JL_ERR_CUDA = 3,        /* a CUDA call failed                                 */
+  JL_ERR_TIMEOUT = 4      /* a bounded in-kernel wait ran out                   */
+} jl_status;
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* jl_last_error(void);
+
+/* G = max(1, ceil(L / w_pretrained)) (Methodology section 1, dynamic grouping).
+ * Host helper; returns -1 if w_pretrained < 1 or L < 0. */
+int64_t jl_group_size(int64_t L, int64_t w_pretrained);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * JL_OK, JL_ERR_TIMEOUT, or JL_ERR_CUDA if the synchronisation itself failed. */
+jl_status jl_sync_status(jl_stream_t stream);
+
+/*
+ * RoPE cos/sin tables.  Fills cos_out[p][c] = cos(p * theta_c) and
+ * sin_out[p][c] = sin(p * theta_c) for p in [0, n_pos), c in [0, head_dim/2),
+ * row-major fp32 [n_pos][head_dim/2].  Angles and cos/sin are computed in fp64
+ * on the device and rounded to fp32 once.  Both the base rotations R(i) and the
+ * remote rotations R(f(i)) read these rows (remote rows are < w_pretrained);
+ * decode also reads rows n = x - f(x) for its correction rotations.
+ * Requirements: n_pos >= 1, head_dim in {64, 128}, rope_base > 1.
+ */
+jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
+                         jl_stream_t stream);
+
+/*
+ * Bifocal prefill (Methodology section 2, inclusion-exclusion attention merge).
+ * Computes, for every token i of every packed sequence and every query head,
+ *   out = softmax_j(scale * s(i, j)) V   over j <= i, with s the routed score,
+ * which equals the inclusion-exclusion merge of the three flash passes
+ * (local/base + causal/remote - local/remote) on their log-sum-exp statistics.
+ *
+ *   q           bf16 [total_tokens][Hq][head_dim], RAW (not rotated)
+ *   k, v        bf16 [total_tokens][Hkv][head_dim], k RAW
+ *   cu_seqlens  device int32 [batch + 1], cu_seqlens[0] = 0, non-decreasing,
+ *               cu_seqlens[batch] = total_tokens.  Positions restart at 0 in
+ *               every sequence; G is computed per sequence from its length.
+ *   max_seqlen  >= every sequence length (sizes the grid)
+ *   w0          >= 0 (0 = no local window); w_pretrained >= 1
+ *   cos_tab, sin_tab  from jl_rope_tables with n_tab_rows >= max_seqlen
+ *   softmax_scale     <= 0 selects 1/sqrt(head_dim)
+ *   out         bf16 [total_tokens][Hq][head_dim]
+ *   lse         fp32 [Hq][total_tokens], natural-log log-sum-exp of the scaled
+ *               routed scores of each row; may be NULL.
+ * Supported: head_dim in {64, 128}; Hq % Hkv == 0; batch >= 0 (0 is a no-op).
+ * No workspace; the kernel keeps everything in shared and tensor memory.
+ */
+jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                             int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                             int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                             const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
+                             jl_stream_t stream);
+
+/* Plain causal RoPE prefill (every causal pair LOCAL), built from the same
+ * kernel; the comparator for bifocal prefill.  Same conventions. */
+jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                           int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,
+                           void* out, float* lse, jl_stream_t stream);
+
+/*
+ * Single-query bifocal decode with the on-the-fly correction rotation
+ * (Methodology section 2).  One new token per batch entry b sits at position
+ * i = seqlens[b] - 1 of a base-RoPE KV cache.
+ *
+ *   q            bf16 [B][Hq][head_dim], ALREADY rotated by R(i) (base RoPE)
+ *   k_cache      bf16 [B][cache_stride][Hkv][head_dim]: keys rotated by R(j)
+ *                at their absolute positions j; the caller has already
+ *                appended the current token.  READ ONLY: never written.
+ *   v_cache      bf16 [B][cache_stride][Hkv][head_dim], read only
+ *   seqlens      device int32 [B], 1 <= seqlens[b] <= max_seqlen
+ *   max_seqlen   <= cache_stride; sizes the split-K grid (the call does not
+ *                read seqlens on the host, so it can be captured in a CUDA
+ *                graph and replayed across G changes)
+ *   cos_tab, sin_tab  from jl_rope_tables, n_tab_rows >= max_seqlen
+ *   out          bf16 [B][Hq][head_dim]
+ *   lse          fp32 [B][Hq] natural-log LSE; may be NULL
+ *   workspace    device scratch of at least jl_bifocal_decode_workspace_size()
+ *                bytes, 16-byte aligned, owned by the caller; its contents on
+ *                entry do not matter; calls sharing it must not overlap.
+ * Local keys (i - j < w0) score q . k_cache[j] unchanged; remote keys score
+ * (R(f(i) - i) q) . (R(f(j) - j) k_cache[j]), both corrections applied in
+ * registers.  G = max(1, ceil(seqlens[b] / w_pretrained)) is computed on the
+ * device every call.
+ */
+jl_status jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                            int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                            int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                            const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, jl_stream_t stream);
+
+/* Bytes of workspace jl_bifocal_decode / jl_plain_decode need for these sizes. */
+size_t jl_bifocal_decode_workspace_size(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen);
+
+/* Plain causal decode (no correction rotation), built from the same kernel;
+ * the comparator for the decode overhead.  Same conventions. */
+jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                          int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                          int32_t head_dim, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                          float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                          jl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* JETLONG_H */

@@ -99,6 +99,29 @@ void jlo_rotate(const double* x, int32_t d, int64_t pos, double rope_base, doubl
   free(theta);
 }
 
+void jlo_rotate_rows(const double* x, const int64_t* pos, int64_t n, int32_t d, double rope_base, double* y) {
+  int32_t h = d / 2;
+  double* theta = (double*)malloc(sizeof(double) * (size_t)h);
+  jlo_inv_freq(d, rope_base, theta);
+#pragma omp parallel
+  {
+    double* cs = (double*)malloc(sizeof(double) * (size_t)h * 2);
+    double* sn = cs + h;
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+      int64_t m = pos[r] < 0 ? -pos[r] : pos[r];
+      for (int32_t c = 0; c < h; ++c) {
+        double a = (double)m * theta[c];
+        cs[c] = cos(a);
+        sn[c] = sin(a);
+      }
+      rotate_with(x + r * d, d, cs, sn, pos[r] < 0 ? -1.0 : 1.0, y + r * d);
+    }
+    free(cs);
+  }
+  free(theta);
+}
+
 static double dot(const double* a, const double* b, int32_t d) {
   double s = 0.0;
   for (int32_t c = 0; c < d; ++c) s += a[c] * b[c];

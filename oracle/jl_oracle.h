@@ -65,6 +65,9 @@ void jlo_rope_cos_sin(int64_t n_pos, int32_t d, double rope_base, double* cos_ou
 /* y = R(pos) x, rotate-half convention; pos may be negative (R(-n) = R(n)^T). */
 void jlo_rotate(const double* x, int32_t d, int64_t pos, double rope_base, double* y);
 
+/* y_r = R(pos_r) x_r for n rows of width d (x, y: [n][d] fp64; pos may be negative). */
+void jlo_rotate_rows(const double* x, const int64_t* pos, int64_t n, int32_t d, double rope_base, double* y);
+
 /*
  * Direct definition for one sequence of length L.  For each selected row r
  * (query position i = row_pos[r], query head h = row_head[r]) build the

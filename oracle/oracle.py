@@ -48,6 +48,8 @@ def lib():
         _lib.jlo_inv_freq.argtypes = [i32, dbl, vp]
         _lib.jlo_rope_cos_sin.restype = None
         _lib.jlo_rope_cos_sin.argtypes = [i64, i32, dbl, vp, vp]
+        _lib.jlo_rotate_rows.restype = None
+        _lib.jlo_rotate_rows.argtypes = [vp, vp, i64, i32, dbl, vp]
         _lib.jlo_rotate.restype = None
         _lib.jlo_rotate.argtypes = [vp, i32, i64, dbl, vp]
         rows_args = [View, View, View, i64, i32, i32, i32, vp, vp, i64, i64, i64, dbl, dbl]
@@ -103,6 +105,16 @@ def rotate(x: np.ndarray, pos: int, base: float) -> np.ndarray:
     x = np.ascontiguousarray(x, np.float64)
     y = np.zeros_like(x)
     lib().jlo_rotate(_ptr(x), x.shape[-1], pos, base, _ptr(y))
+    return y
+
+
+def rotate_rows(x: np.ndarray, pos: np.ndarray, base: float) -> np.ndarray:
+    """R(pos[r]) x[r] for x [n][d] (any float dtype, upcast to fp64)."""
+    x = np.ascontiguousarray(x, np.float64)
+    n, d = x.shape
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, np.int64), (n,)))
+    y = np.empty_like(x)
+    lib().jlo_rotate_rows(_ptr(x), _ptr(p), n, d, base, _ptr(y))
     return y
 
 

@@ -1,0 +1,48 @@
+"""Build libjetlong.so in-tree with nvcc for sm_100a (B200).
+
+``python -m rope_context_extension_sm_b200.build`` compiles the single
+translation unit ``csrc/jetlong.cu`` (which includes the kernel headers) into
+``rope_context_extension_sm_b200/libjetlong.so``.  nvcc cross-compiles, so this
+also works on a machine without a GPU.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libjetlong.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+FLAGS = [
+    "-O3", "-std=c++17", "-lineinfo",
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-Xcompiler", "-fPIC,-O2,-Wall",
+    "--expt-relaxed-constexpr",
+    "-shared",
+]
+
+
+def sources() -> list[str]:
+    return sorted(glob.glob(os.path.join(CSRC, "*")) + [os.path.join(ROOT, "include", "jetlong.h")])
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    newest = max(os.path.getmtime(p) for p in sources())
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not extra:
+        return LIB
+    cmd = [NVCC, *FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"), "-I", CSRC,
+           "-o", LIB, os.path.join(CSRC, "jetlong.cu")]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.run(cmd, check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose=True, extra=sys.argv[1:])
+    print(LIB)

@@ -1,0 +1,328 @@
+// jetlong.cu -- the C ABI of libjetlong.so (declared in include/jetlong.h):
+// argument validation, TMA tensor-map encoding and kernel launches for the
+// bifocal prefill, the split-K bifocal decode, their plain comparators and the
+// RoPE tables.  One translation unit, so the device status word needs no
+// relocatable device code.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "jetlong.h"
+#include "jl_decode.cuh"
+#include "jl_prefill.cuh"
+#include "jl_tables.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+jl_status fail(jl_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+jl_status fail(jl_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+jl_status ok() {
+  g_err.clear();
+  return JL_OK;
+}
+
+jl_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(JL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- TMA maps --
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [tokens][heads][d] bf16, box = 64 channels x 1 head x 128 tokens, 128B swizzle.
+jl_status make_map(CUtensorMap* map, const void* base, int64_t tokens, int heads, int d) {
+  auto fn = encode_fn();
+  if (!fn) return fail(JL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(heads) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(JL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return JL_OK;
+}
+
+// ----------------------------------------------------------------- prefill --
+
+template <int D, int NQT>
+jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::PrefillParams& prm,
+                         cudaStream_t st) {
+  using Lay = jl::PrefillLayout<D, NQT>;
+  CUtensorMap tq, tk, tv;
+  jl_status s;
+  if ((s = make_map(&tq, q, prm.total_tokens, prm.Hq, D)) != JL_OK) return s;
+  if ((s = make_map(&tk, k, prm.total_tokens, prm.Hkv, D)) != JL_OK) return s;
+  if ((s = make_map(&tv, v, prm.total_tokens, prm.Hkv, D)) != JL_OK) return s;
+  auto kern = jl::jl_prefill_kernel<D, NQT>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
+  const int64_t blocks = static_cast<int64_t>(prm.n_qtiles) * prm.batch * prm.Hkv * prm.slots;
+  if (blocks > 0x7fffffff) return fail(JL_ERR_UNSUPPORTED, "prefill grid too large (%lld blocks)", (long long)blocks);
+  kern<<<static_cast<unsigned>(blocks), Lay::kThreads, Lay::kAlloc, st>>>(tq, tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
+jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                         int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                         int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
+                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, cudaStream_t st) {
+  if (batch < 0) return fail(JL_ERR_INVALID, "batch must be >= 0 (got %d)", batch);
+  if (total_tokens < 0 || total_tokens > 0x7fffffffLL)
+    return fail(JL_ERR_INVALID, "total_tokens must be in [0, 2^31) (got %lld)", (long long)total_tokens);
+  if (max_seqlen < 0) return fail(JL_ERR_INVALID, "max_seqlen must be >= 0 (got %d)", max_seqlen);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(JL_ERR_INVALID, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (got Hq=%d, Hkv=%d)", Hq, Hkv);
+  if (w0 < 0) return fail(JL_ERR_INVALID, "w0 must be >= 0 (got %d)", w0);
+  if (w_pretrained < 1) return fail(JL_ERR_INVALID, "w_pretrained must be >= 1 (got %d)", w_pretrained);
+  if (batch == 0 || total_tokens == 0 || max_seqlen == 0) return ok();
+  if (!q || !k || !v || !cu_seqlens || !cos_tab || !sin_tab || !out)
+    return fail(JL_ERR_INVALID, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cos_tab) ||
+      !aligned16(sin_tab))
+    return fail(JL_ERR_INVALID, "q, k, v, out and the tables must be 16-byte aligned");
+  if (n_tab_rows < max_seqlen)
+    return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_seqlen (%d)", (long long)n_tab_rows, max_seqlen);
+  jl::PrefillParams prm{};
+  prm.cu_seqlens = cu_seqlens;
+  prm.cos_tab = cos_tab;
+  prm.sin_tab = sin_tab;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.total_tokens = total_tokens;
+  prm.n_tab_rows = n_tab_rows;
+  prm.batch = batch;
+  prm.n_qtiles = (max_seqlen + jl::kBM - 1) / jl::kBM;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.w0 = w0;
+  prm.w_pre = w_pretrained;
+  prm.plain = plain;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const bool pair = (prm.group % 2) == 0;
+  prm.slots = prm.group / (pair ? 2 : 1);
+  if (head_dim == 128)
+    return pair ? launch_prefill<128, 2>(q, k, v, prm, st) : launch_prefill<128, 1>(q, k, v, prm, st);
+  return pair ? launch_prefill<64, 2>(q, k, v, prm, st) : launch_prefill<64, 1>(q, k, v, prm, st);
+}
+
+// ------------------------------------------------------------------ decode --
+
+int decode_chunk(int32_t max_seqlen) {
+  int c = 64;
+  while (c < 512 && static_cast<int64_t>(c) * 256 < max_seqlen) c *= 2;
+  return c;
+}
+
+template <int D, int GROUP, bool PLAIN>
+jl_status launch_decode(const jl::DecodeParams& prm, int B, cudaStream_t st) {
+  dim3 grid(prm.Hkv, prm.n_split, B);
+  jl::jl_decode_split_kernel<D, GROUP, PLAIN><<<grid, jl::kDecodeThreads, 0, st>>>(prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  jl::jl_decode_combine_kernel<D><<<dim3(prm.Hq, B), D, 0, st>>>(prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return ok();
+}
+
+template <int D, bool PLAIN>
+jl_status dispatch_group(const jl::DecodeParams& prm, int B, cudaStream_t st) {
+  switch (prm.group) {
+    case 1: return launch_decode<D, 1, PLAIN>(prm, B, st);
+    case 2: return launch_decode<D, 2, PLAIN>(prm, B, st);
+    case 4: return launch_decode<D, 4, PLAIN>(prm, B, st);
+    case 8: return launch_decode<D, 8, PLAIN>(prm, B, st);
+    default: return fail(JL_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8} (got %d)", prm.group);
+  }
+}
+
+size_t decode_ws_bytes(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {
+  if (B <= 0 || Hq <= 0 || head_dim <= 0 || max_seqlen <= 0) return 0;
+  const int chunk = decode_chunk(max_seqlen);
+  const int64_t n_split = (max_seqlen + chunk - 1) / chunk;
+  return static_cast<size_t>(B) * n_split * Hq * (head_dim + 2) * sizeof(float);
+}
+
+jl_status decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int32_t B,
+                        int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                        int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
+                        int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                        size_t workspace_bytes, cudaStream_t st) {
+  if (B < 0) return fail(JL_ERR_INVALID, "B must be >= 0 (got %d)", B);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(JL_ERR_INVALID, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (got Hq=%d, Hkv=%d)", Hq, Hkv);
+  if (w0 < 0) return fail(JL_ERR_INVALID, "w0 must be >= 0 (got %d)", w0);
+  if (w_pretrained < 1) return fail(JL_ERR_INVALID, "w_pretrained must be >= 1 (got %d)", w_pretrained);
+  if (B == 0) return ok();
+  if (max_seqlen < 1) return fail(JL_ERR_INVALID, "max_seqlen must be >= 1 (got %d)", max_seqlen);
+  if (cache_stride < max_seqlen)
+    return fail(JL_ERR_INVALID, "cache_stride (%lld) must be >= max_seqlen (%d)", (long long)cache_stride,
+                max_seqlen);
+  if (n_tab_rows < max_seqlen)
+    return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_seqlen (%d)", (long long)n_tab_rows, max_seqlen);
+  if (!q || !k_cache || !v_cache || !seqlens || !cos_tab || !sin_tab || !out || !workspace)
+    return fail(JL_ERR_INVALID, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace) ||
+      !aligned16(cos_tab) || !aligned16(sin_tab))
+    return fail(JL_ERR_INVALID, "q, caches, out, workspace and the tables must be 16-byte aligned");
+  const size_t need = decode_ws_bytes(B, Hq, head_dim, max_seqlen);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  jl::DecodeParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k_cache);
+  prm.v = static_cast<const __nv_bfloat16*>(v_cache);
+  prm.seqlens = seqlens;
+  prm.cos_tab = cos_tab;
+  prm.sin_tab = sin_tab;
+  prm.ws = static_cast<float*>(workspace);
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.cache_stride = cache_stride;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.w0 = w0;
+  prm.w_pre = w_pretrained;
+  prm.plain = plain;
+  prm.chunk = decode_chunk(max_seqlen);
+  prm.n_split = (max_seqlen + prm.chunk - 1) / prm.chunk;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  if (head_dim == 128)
+    return plain ? dispatch_group<128, true>(prm, B, st) : dispatch_group<128, false>(prm, B, st);
+  return plain ? dispatch_group<64, true>(prm, B, st) : dispatch_group<64, false>(prm, B, st);
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+
+extern "C" {
+
+const char* jl_last_error(void) { return g_err.c_str(); }
+
+int64_t jl_group_size(int64_t L, int64_t w_pretrained) {
+  if (w_pretrained < 1 || L < 0) return -1;
+  const int64_t g = (L + w_pretrained - 1) / w_pretrained;
+  return g < 1 ? 1 : g;
+}
+
+jl_status jl_sync_status(jl_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, jl::g_status, sizeof word);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (word != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(jl::g_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    if (word & jl::kDevErrTimeout) return fail(JL_ERR_TIMEOUT, "a bounded in-kernel wait ran out");
+  }
+  return ok();
+}
+
+jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
+                         jl_stream_t stream) {
+  if (!cos_out || !sin_out) return fail(JL_ERR_INVALID, "null table pointer");
+  if (n_pos < 1) return fail(JL_ERR_INVALID, "n_pos must be >= 1 (got %lld)", (long long)n_pos);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (!(rope_base > 1.0)) return fail(JL_ERR_INVALID, "rope_base must be > 1");
+  if (!aligned16(cos_out) || !aligned16(sin_out)) return fail(JL_ERR_INVALID, "tables must be 16-byte aligned");
+  const int half = head_dim / 2;
+  const int64_t total = n_pos * half;
+  const int64_t blocks64 = (total + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(blocks64 < 148 * 64 ? blocks64 : 148 * 64);
+  jl::jl_rope_table_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cos_out, sin_out, n_pos,
+                                                                                       half, rope_base);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rope table launch");
+  return ok();
+}
+
+jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                             int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                             int32_t w0, int32_t w_pretrained, const float* cos_tab, const float* sin_tab,
+                             int64_t n_tab_rows, float softmax_scale, void* out, float* lse, jl_stream_t stream) {
+  return prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0, w_pretrained,
+                        0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                           int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                           const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,
+                           void* out, float* lse, jl_stream_t stream) {
+  return prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, 0, 1, 1, cos_tab,
+                        sin_tab, n_tab_rows, softmax_scale, out, lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t jl_bifocal_decode_workspace_size(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {
+  return decode_ws_bytes(B, Hq, head_dim, max_seqlen);
+}
+
+jl_status jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                            int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                            int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                            const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, jl_stream_t stream) {
+  return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim, w0,
+                       w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, workspace,
+                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int32_t B,
+                          int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                          const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,
+                          void* out, float* lse, void* workspace, size_t workspace_bytes, jl_stream_t stream) {
+  return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim, 0, 1, 1,
+                       cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

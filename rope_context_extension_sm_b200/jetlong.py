@@ -1,0 +1,212 @@
+"""Thin ctypes binding of libjetlong.so (C ABI in include/jetlong.h).
+
+Argument marshalling only: every function checks tensor dtypes, devices and
+shapes, allocates outputs with torch when the caller passes none, and forwards
+raw device pointers plus the current CUDA stream to the C entry point of the
+same name.  All attention arithmetic runs in the library's CUDA kernels; there
+is no CPU fallback.  Importing this module loads the library and raises
+``ImportError`` if it has not been built (``python -m
+rope_context_extension_sm_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjetlong.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libjetlong.so is not built ({LIB_PATH}); run python -m rope_context_extension_sm_b200.build")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+JL_OK, JL_ERR_INVALID, JL_ERR_UNSUPPORTED, JL_ERR_CUDA, JL_ERR_TIMEOUT = range(5)
+_NAMES = {0: "JL_OK", 1: "JL_ERR_INVALID", 2: "JL_ERR_UNSUPPORTED", 3: "JL_ERR_CUDA", 4: "JL_ERR_TIMEOUT"}
+
+_vp, _i32, _i64, _f32, _f64, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                    ctypes.c_double, ctypes.c_size_t)
+
+# Every symbol include/jetlong.h declares, with its C signature.
+SIGNATURES = {
+    "jl_last_error": (ctypes.c_char_p, []),
+    "jl_group_size": (_i64, [_i64, _i64]),
+    "jl_sync_status": (ctypes.c_int, [_vp]),
+    "jl_rope_tables": (ctypes.c_int, [_vp, _vp, _i64, _i32, _f64, _vp]),
+    "jl_bifocal_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
+                                          _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
+    "jl_plain_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
+                                        _f32, _vp, _vp, _vp]),
+    "jl_bifocal_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
+                                         _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "jl_bifocal_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "jl_plain_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
+                                       _f32, _vp, _vp, _vp, _sz, _vp]),
+}
+
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class JetLongError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.jl_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != JL_OK:
+        raise JetLongError(status, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: int | None = None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions (got {t.dim()})")
+
+
+def jl_last_error() -> str:
+    return _lib.jl_last_error().decode(errors="replace")
+
+
+def jl_group_size(L: int, w_pretrained: int) -> int:
+    return int(_lib.jl_group_size(L, w_pretrained))
+
+
+def jl_sync_status(stream=None) -> None:
+    """Synchronise the stream and raise JetLongError if a kernel's bounded wait ran out."""
+    _check(_lib.jl_sync_status(_stream(stream)), "jl_sync_status")
+
+
+def jl_rope_tables(n_pos: int, head_dim: int, rope_base: float, *, device="cuda", cos=None, sin=None, stream=None):
+    """fp32 [n_pos][head_dim/2] cos/sin tables (allocated unless given)."""
+    if cos is None:
+        cos = torch.empty((n_pos, head_dim // 2), dtype=torch.float32, device=device)
+    if sin is None:
+        sin = torch.empty((n_pos, head_dim // 2), dtype=torch.float32, device=device)
+    _need(cos, torch.float32, "cos", 2)
+    _need(sin, torch.float32, "sin", 2)
+    _check(_lib.jl_rope_tables(_ptr(cos), _ptr(sin), n_pos, head_dim, float(rope_base), _stream(stream)),
+           "jl_rope_tables")
+    return cos, sin
+
+
+def _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse):
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k, torch.bfloat16, "k", 3)
+    _need(v, torch.bfloat16, "v", 3)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
+    _need(cos, torch.float32, "cos", 2)
+    _need(sin, torch.float32, "sin", 2)
+    T, hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != T or k.shape[2] != d:
+        raise ValueError("k and v must be [T][Hkv][d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.bfloat16, "out", 3)
+    if lse is None and want_lse:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", 2)
+    return T, hq, k.shape[1], d, out, lse
+
+
+def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, *,
+                       softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True, stream=None):
+    """Bifocal prefill over packed sequences. q [T][Hq][d], k/v [T][Hkv][d] raw bf16.
+
+    Returns (out bf16 [T][Hq][d], lse fp32 [Hq][T] or None)."""
+    T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
+    batch = cu_seqlens.shape[0] - 1
+    _check(_lib.jl_bifocal_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq, hkv, d,
+                                   w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out),
+                                   _ptr(lse), _stream(stream)), "jl_bifocal_prefill")
+    return out, lse
+
+
+def jl_plain_prefill(q, k, v, cu_seqlens, max_seqlen: int, cos, sin, *, softmax_scale: float = 0.0, out=None,
+                     lse=None, want_lse: bool = True, stream=None):
+    """Plain causal RoPE prefill (comparator), same layout as jl_bifocal_prefill."""
+    T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
+    batch = cu_seqlens.shape[0] - 1
+    _check(_lib.jl_plain_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq, hkv, d,
+                                 _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out), _ptr(lse),
+                                 _stream(stream)), "jl_plain_prefill")
+    return out, lse
+
+
+def jl_bifocal_decode_workspace_size(B: int, Hq: int, head_dim: int, max_seqlen: int) -> int:
+    return int(_lib.jl_bifocal_decode_workspace_size(B, Hq, head_dim, max_seqlen))
+
+
+def _decode_args(q, k_cache, v_cache, seqlens, cos, sin, max_seqlen, out, lse, workspace, want_lse):
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(seqlens, torch.int32, "seqlens", 1)
+    _need(cos, torch.float32, "cos", 2)
+    _need(sin, torch.float32, "sin", 2)
+    B, hq, d = q.shape
+    if k_cache.shape != v_cache.shape or k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError("k_cache and v_cache must be [B][cache_stride][Hkv][d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    need = jl_bifocal_decode_workspace_size(B, hq, d, max_seqlen)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    return B, hq, k_cache.shape[2], d, out, lse, workspace
+
+
+def jl_bifocal_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, *,
+                      softmax_scale: float = 0.0, out=None, lse=None, workspace=None, want_lse: bool = True,
+                      stream=None):
+    """Single-query bifocal decode on a base-RoPE cache (cache is only read).
+
+    q [B][Hq][d] already rotated by R(seqlens[b]-1); caches [B][stride][Hkv][d].
+    Returns (out bf16 [B][Hq][d], lse fp32 [B][Hq] or None)."""
+    B, hq, hkv, d, out, lse, ws = _decode_args(q, k_cache, v_cache, seqlens, cos, sin, max_seqlen, out, lse,
+                                               workspace, want_lse)
+    _check(_lib.jl_bifocal_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, k_cache.shape[1],
+                                  max_seqlen, hq, hkv, d, w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0],
+                                  softmax_scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "jl_bifocal_decode")
+    return out, lse
+
+
+def jl_plain_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, cos, sin, *, softmax_scale: float = 0.0,
+                    out=None, lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """Plain causal decode (comparator), same layout as jl_bifocal_decode."""
+    B, hq, hkv, d, out, lse, ws = _decode_args(q, k_cache, v_cache, seqlens, cos, sin, max_seqlen, out, lse,
+                                               workspace, want_lse)
+    _check(_lib.jl_plain_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, k_cache.shape[1],
+                                max_seqlen, hq, hkv, d, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale,
+                                _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "jl_plain_decode")
+    return out, lse
+
+
+def default_scale(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on the
+same seeded bf16 inputs.
+
+Acceptance (bf16 inputs, fp32 accumulation): output max-abs <= 2e-2, output
+mean-abs <= 2e-3, LSE max-abs <= 1e-2.  Small cases compare every row; the
+model-sized cases compare sampled rows plus the critical rows (window edge,
+pretraining-window edge, tile edges, last rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from rope_context_extension_sm_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module")
+def jl():
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    from rope_context_extension_sm_b200 import build
+    build.build()
+    from rope_context_extension_sm_b200 import jetlong
+    return jetlong
+
+
+def _tables(jl, n, d, base):
+    return jl.jl_rope_tables(n, d, base)
+
+
+def _check(got_out, got_lse, ref_out, ref_lse, what):
+    err = np.abs(got_out.astype(np.float64) - ref_out)
+    lerr = np.abs(got_lse.astype(np.float64) - ref_lse)
+    assert np.isfinite(got_out).all() and np.isfinite(got_lse).all(), what
+    assert err.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e}"
+    assert err.mean() <= OUT_MEAN, f"{what}: out mean-abs {err.mean():.3e}"
+    assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
+    return err.max(), err.mean(), lerr.max()
+
+
+def _prefill_gpu(jl, q, k, v, cu, cfg, plain=False):
+    dev = "cuda"
+    qd, kd, vd, cud = q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
+    cos, sin = _tables(jl, max(cfg.max_seqlen, 1), cfg.head_dim, cfg.rope_base)
+    if plain:
+        out, lse = jl.jl_plain_prefill(qd, kd, vd, cud, cfg.max_seqlen, cos, sin)
+    else:
+        out, lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, cfg.w0, cfg.w_pretrained, cos, sin)
+    jl.jl_sync_status()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _oracle_rows(q, k, v, cu, cfg, seq, rows, heads, plain=False):
+    s0, s1 = int(cu[seq]), int(cu[seq + 1])
+    qb, kb, vb = I.bf16_bits(q[s0:s1]), I.bf16_bits(k[s0:s1]), I.bf16_bits(v[s0:s1])
+    return O.bifocal_rows(qb, kb, vb, s1 - s0, rows, heads, w0=cfg.w0, w_pretrained=cfg.w_pretrained,
+                          rope_base=cfg.rope_base, plain=plain)
+
+
+def _compare_all_rows(jl, cfg, plain=False):
+    q, k, v, cu = I.prefill_inputs(cfg)
+    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg, plain)
+    for s in range(len(cfg.seqlens)):
+        L = cfg.seqlens[s]
+        if L == 0:
+            continue
+        pos = np.repeat(np.arange(L), cfg.n_q_heads)
+        head = np.tile(np.arange(cfg.n_q_heads), L)
+        ro, rl = _oracle_rows(q, k, v, cu, cfg, s, pos, head, plain)
+        s0 = int(cu[s])
+        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{cfg.name} seq {s}")
+    return out, lse
+
+
+# ------------------------------------------------------------------ tables ----
+
+@pytest.mark.parametrize("n,d,base", [(256, 64, 1e4), (131072, 128, 1e6)])
+def test_rope_tables_match_fp64_rounded_once(jl, n, d, base):
+    cos, sin = _tables(jl, n, d, base)
+    jl.jl_sync_status()
+    rc, rs = O.rope_cos_sin(n, d, base)
+    for got, ref in ((cos, rc), (sin, rs)):
+        g = got.cpu().numpy()
+        r32 = ref.astype(np.float32)
+        ulps = np.abs(g.view(np.int32).astype(np.int64) - r32.view(np.int32).astype(np.int64))
+        assert ulps.max() <= 1, f"table differs from fp64-rounded by {ulps.max()} ulp"
+        assert (ulps > 0).mean() < 1e-3
+
+
+# ----------------------------------------------------------------- prefill ----
+
+def test_tiny_prefill_all_rows(jl):
+    """L = 256, d = 64, G = 4, w0 = 32: every row against the oracle."""
+    _compare_all_rows(jl, I.TINY)
+
+
+def test_tiny_plain_prefill_all_rows(jl):
+    _compare_all_rows(jl, I.TINY, plain=True)
+
+
+SMALL = [
+    # name, seqlens, Hq, Hkv, d, w0, w_pre
+    ("gqa4_G4_w0_100", (1000,), 8, 2, 128, 100, 256),
+    ("gqa4_G4_w0_0", (1000,), 8, 2, 128, 0, 256),
+    ("gqa4_G4_w0_1", (1000,), 8, 2, 128, 1, 256),
+    ("gqa4_G4_w0_127", (777,), 4, 1, 128, 127, 200),
+    ("gqa4_G4_w0_128", (777,), 4, 1, 128, 128, 200),
+    ("gqa4_G4_w0_129", (777,), 4, 1, 128, 129, 200),
+    ("gqa2_G3_w0_300", (700,), 4, 2, 128, 300, 256),
+    ("w0_covers_all", (600,), 4, 2, 128, 5000, 100),
+    ("G1_short", (300,), 4, 2, 128, 64, 512),
+    ("varlen_ragged", (1, 130, 257, 700, 64, 129), 4, 2, 128, 50, 128),
+    ("group3_d64", (500,), 3, 1, 64, 40, 100),
+    ("group1_d128", (384,), 2, 2, 128, 64, 100),
+    ("d64_gqa2", (450,), 4, 2, 64, 33, 64),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_prefill_all_rows(jl, case):
+    name, seqlens, hq, hkv, d, w0, w_pre = case
+    cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
+    _compare_all_rows(jl, cfg)
+
+
+def test_short_input_gpu_bifocal_equals_plain_bitwise(jl):
+    """L <= w_pretrained (G = 1): the kernel takes the plain path, so the outputs are identical."""
+    cfg = I.PrefillConfig("G1", (900,), 8, 2, 128, 100, 1024, 1e6, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    ob, lb = _prefill_gpu(jl, q, k, v, cu, cfg)
+    op, lp = _prefill_gpu(jl, q, k, v, cu, cfg, plain=True)
+    np.testing.assert_array_equal(ob, op)
+    np.testing.assert_array_equal(lb, lp)
+
+
+def test_empty_and_zero_length_sequences(jl):
+    cfg = I.PrefillConfig("with_empty", (0, 200, 0, 5), 2, 1, 128, 16, 64, 1e4, False)
+    _compare_all_rows(jl, cfg)
+
+
+def _critical_rows(L, w0, w_pre, extra_seed, n_random):
+    rows = {0, 1, 2, 126, 127, 128, 129, w0 - 2, w0 - 1, w0, w0 + 1, w0 + 127, w0 + 128, w_pre - 1, w_pre,
+            w_pre + 1, L - 129, L - 128, L - 2, L - 1}
+    rng = np.random.default_rng(extra_seed)
+    rows |= set(rng.integers(0, L, n_random).tolist())
+    return sorted(r for r in rows if 0 <= r < L)
+
+
+def _compare_sampled(jl, cfg, n_random=24, heads_per_row=4, seed=11):
+    q, k, v, cu = I.prefill_inputs(cfg)
+    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg)
+    rng = np.random.default_rng(seed)
+    worst = (0.0, 0.0, 0.0)
+    for s in range(len(cfg.seqlens)):
+        L = cfg.seqlens[s]
+        rows = _critical_rows(L, cfg.w0, cfg.w_pretrained, seed + s, n_random)
+        pos, head = [], []
+        for r in rows:
+            hs = rng.choice(cfg.n_q_heads, size=min(heads_per_row, cfg.n_q_heads), replace=False)
+            pos += [r] * len(hs)
+            head += hs.tolist()
+        pos, head = np.array(pos), np.array(head)
+        ro, rl = _oracle_rows(q, k, v, cu, cfg, s, pos, head)
+        s0 = int(cu[s])
+        e = _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{cfg.name} seq {s}")
+        worst = tuple(max(a, b) for a, b in zip(worst, e))
+    assert np.isfinite(out).all()
+    return worst
+
+
+@pytest.mark.parametrize("w0", I.W0_SWEEP)
+def test_qwen3_1p7b_64k_sampled_rows(jl, w0):
+    _compare_sampled(jl, I.with_(I.QWEN3_1P7B, w0=w0), n_random=12 if w0 != 4096 else 24)
+
+
+def test_qwen3_8b_128k_sampled_rows(jl):
+    _compare_sampled(jl, I.QWEN3_8B_128K, n_random=24)
+
+
+@pytest.mark.parametrize("L", [32768, 32769])
+def test_group_boundary_32768(jl, L):
+    """G jumps from 1 to 2 between L = 32768 and L = 32769."""
+    _compare_sampled(jl, I.with_(I.QWEN3_8B_128K, seqlens=(L,)), n_random=8)
+
+
+def test_varlen_sampled_rows(jl):
+    _compare_sampled(jl, I.VARLEN, n_random=6, heads_per_row=2)
+
+
+# ------------------------------------------------------------------ decode ----
+
+def _decode_setup(cfg, max_len, batch=1):
+    """Raw keys -> base-RoPE cache k~_j = bf16(R(j) k_j) (rotated by the oracle in fp64)."""
+    k_raw, v = I.decode_raw_inputs(cfg, max_len, batch)
+    d = cfg.head_dim
+    kr = k_raw.float().numpy().reshape(batch, max_len, cfg.n_kv_heads, d)
+    pos = np.broadcast_to(np.arange(max_len)[None, :, None], (batch, max_len, cfg.n_kv_heads)).reshape(-1)
+    kc = O.rotate_rows(kr.reshape(-1, d), pos, cfg.rope_base).reshape(batch, max_len, cfg.n_kv_heads, d)
+    k_cache = torch.from_numpy(kc).to(torch.bfloat16)
+    return k_cache, v
+
+
+def _query_tilde(cfg, q_raw, L):
+    """bf16(R(L-1) q) for q_raw [Hq][d] bf16."""
+    qt = O.rotate_rows(q_raw.float().numpy(), np.full(q_raw.shape[0], L - 1), cfg.rope_base)
+    return torch.from_numpy(qt).to(torch.bfloat16)
+
+
+def _decode_oracle(cfg, q_t, k_cache_b, v_b, L, plain=False):
+    return O.decode_step(I.bf16_bits(q_t), I.bf16_bits(k_cache_b[:L]), I.bf16_bits(v_b[:L]), L, w0=cfg.w0,
+                         w_pretrained=cfg.w_pretrained, rope_base=cfg.rope_base, plain=plain)
+
+
+def _run_decode(jl, cfg, q_t, k_cache_d, v_d, seqlens, max_len, cos, sin, plain=False):
+    sl = torch.tensor(seqlens, dtype=torch.int32, device="cuda")
+    if plain:
+        out, lse = jl.jl_plain_decode(q_t.cuda(), k_cache_d, v_d, sl, max_len, cos, sin)
+    else:
+        out, lse = jl.jl_bifocal_decode(q_t.cuda(), k_cache_d, v_d, sl, max_len, cfg.w0, cfg.w_pretrained, cos,
+                                        sin)
+    jl.jl_sync_status()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+SMALL_DECODE = I.DecodeConfig("small_decode", (), 8, 2, 128, 100, 256, 1e4)
+
+
+@pytest.mark.parametrize("L", [1, 2, 100, 101, 255, 256, 257, 700, 1000, 1024])
+def test_small_decode_steps(jl, L):
+    cfg = SMALL_DECODE
+    max_len = 1024
+    k_cache, v = _decode_setup(cfg, max_len)
+    q_raw = I.decode_queries(cfg, 1)[0, 0]
+    q_t = _query_tilde(cfg, q_raw, L)
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    out, lse = _run_decode(jl, cfg, q_t[None], k_cache.cuda(), v.cuda(), [L], max_len, cos, sin)
+    ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
+    _check(out[0], lse[0], ro, rl, f"decode L={L}")
+    out, lse = _run_decode(jl, cfg, q_t[None], k_cache.cuda(), v.cuda(), [L], max_len, cos, sin, plain=True)
+    ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L, plain=True)
+    _check(out[0], lse[0], ro, rl, f"plain decode L={L}")
+
+
+def test_batched_decode_each_sequence_its_own_G(jl):
+    cfg = SMALL_DECODE
+    max_len, lens = 1024, [1024, 250, 513, 7]
+    k_cache, v = _decode_setup(cfg, max_len, batch=len(lens))
+    qs = I.decode_queries(cfg, 1, batch=len(lens))[0]
+    q_t = torch.stack([_query_tilde(cfg, qs[b], lens[b]) for b in range(len(lens))])
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    out, lse = _run_decode(jl, cfg, q_t, k_cache.cuda(), v.cuda(), lens, max_len, cos, sin)
+    for b, L in enumerate(lens):
+        ro, rl = _decode_oracle(cfg, q_t[b], k_cache[b], v[b], L)
+        _check(out[b], lse[b], ro, rl, f"batched decode b={b} L={L}")
+
+
+@pytest.mark.parametrize("L", I.DECODE_QWEN3_4B.cache_lens)
+def test_decode_qwen3_4b_cache_lengths(jl, L):
+    cfg = I.DECODE_QWEN3_4B
+    k_cache, v = _decode_setup(cfg, L)
+    q_raw = I.decode_queries(cfg, 1)[0, 0]
+    q_t = _query_tilde(cfg, q_raw, L)
+    cos, sin = _tables(jl, L, cfg.head_dim, cfg.rope_base)
+    kd, vd = k_cache.cuda(), v.cuda()
+    before = (kd.view(torch.int16).sum(dtype=torch.int64).item(), vd.view(torch.int16).sum(dtype=torch.int64).item())
+    out, lse = _run_decode(jl, cfg, q_t[None], kd, vd, [L], L, cos, sin)
+    after = (kd.view(torch.int16).sum(dtype=torch.int64).item(), vd.view(torch.int16).sum(dtype=torch.int64).item())
+    assert before == after, "the cache must not be written"
+    ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
+    _check(out[0], lse[0], ro, rl, f"decode Qwen3-4B L={L}")
+
+
+def test_decode_walk_across_G_boundary(jl):
+    """Generation across L = 98304 -> 98305 (G 3 -> 4) with no cache rewrite: selected steps of
+    the 256-token walk (positions 98176 .. 98431), all around the boundary."""
+    cfg = I.DECODE_QWEN3_4B
+    first, steps = cfg.walk_first_pos, cfg.walk_steps
+    max_len = first + steps
+    k_cache, v = _decode_setup(cfg, max_len)
+    qs = I.decode_queries(cfg, steps)
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    kd, vd = k_cache.cuda(), v.cuda()
+    chosen = sorted(set(range(124, 132)) | set(range(0, steps, 64)) | {steps - 1})
+    for t in chosen:
+        L = first + t + 1
+        q_t = _query_tilde(cfg, qs[t, 0], L)
+        out, lse = _run_decode(jl, cfg, q_t[None], kd, vd, [L], max_len, cos, sin)
+        ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
+        _check(out[0], lse[0], ro, rl, f"walk step {t} (L={L}, G={O.group_size(L, cfg.w_pretrained)})")

@@ -117,6 +117,14 @@ def test_rotation_matches_complex_multiplication(d, base):
     np.testing.assert_allclose(got, ref, atol=1e-10)
 
 
+def test_rotate_rows_matches_single_rotations():
+    x = _rand((6, 16), 3)
+    pos = np.array([0, 5, -5, 77, 131071, -98303])
+    y = O.rotate_rows(x, pos, 1e6)
+    for r in range(6):
+        np.testing.assert_array_equal(y[r], O.rotate(x[r], int(pos[r]), 1e6))
+
+
 # ---------------------------------------------------- attention helpers ----
 
 def _seq(L, hq, hkv, d, seed):
