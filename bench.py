@@ -1,0 +1,506 @@
+#!/usr/bin/env python
+"""Benchmark of the bifocal attention hot path on B200.
+
+One step = one bifocal prefill of a Qwen3-8B-shaped layer at L = 131072 (32
+query / 8 KV heads, head_dim 128, w_pretrained 32768 -> G = 4, w0 = 4096) plus
+one bifocal decode token against a 131072-token base-RoPE cache (Qwen3-4B
+shape: 32 / 8 heads, head_dim 128).  Inputs are seeded synthetic bf16 data
+(rope_context_extension_sm_b200.inputs), resident in HBM before timing; both
+the prefill inputs (1.5 GB) and the cache (512 MiB) are larger than L2.
+
+Prints ONE JSON line (rank 0).  ``value`` is useful prefill TFLOP/s (each causal
+(q, k) pair counted once at 4 * head_dim flops per query head), aggregated over
+ranks; decode latency, the plain comparators, the roofline of the dominant
+kernel, the end-to-end number through host buffers and the CPU oracle baseline
+ride along in the same line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 (under torchrun) every rank runs an independent replica of the
+step; there is no collective on the data path (the method does not need one).
+``--impl reference`` times the CPU oracle (the only reference implementation
+this method has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rope_context_extension_sm_b200 import inputs as I  # noqa: E402
+
+PREFILL = I.QWEN3_8B_128K
+DECODE = I.DECODE_QWEN3_4B
+DECODE_L = 131072
+METRIC = "bifocal prefill useful TFLOP/s at 128K (frac of BF16 peak); decode us/token"
+UNIT = "TFLOP/s"
+WORKLOAD = "qwen3_8b_prefill_L131072_G4_w0_4096 + qwen3_4b_decode_L131072"
+
+
+def _config():
+    return {
+        "workload": WORKLOAD,
+        "seq_len": PREFILL.seqlens[0],
+        "n_q_heads": PREFILL.n_q_heads,
+        "n_kv_heads": PREFILL.n_kv_heads,
+        "head_dim": PREFILL.head_dim,
+        "w0": PREFILL.w0,
+        "w_pretrained": PREFILL.w_pretrained,
+        "G": I.QWEN3_8B_128K.seqlens[0] // PREFILL.w_pretrained,
+        "decode_cache_len": DECODE_L,
+        "decode_heads": [DECODE.n_q_heads, DECODE.n_kv_heads],
+        "l2": "inputs larger than L2 (prefill 1.5 GB, decode cache 512 MiB); no flush needed",
+        "parallelism": "replicas",
+    }
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+PREFILL_SRC = ["rope_context_extension_sm_b200/csrc/jl_prefill.cuh", "rope_context_extension_sm_b200/csrc/jl_device.cuh"]
+DECODE_SRC = ["rope_context_extension_sm_b200/csrc/jl_decode.cuh", "rope_context_extension_sm_b200/csrc/jl_device.cuh"]
+
+
+def _traffic(kernel, files):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != _source_hash(files):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- our arm ----
+
+def _build_decode_cache(L):
+    """A resident cache of L positions: random bf16 rows stand for base-rotated keys."""
+    k_raw, v = I.decode_raw_inputs(DECODE, L)
+    return k_raw, v
+
+
+def run_ours(args, world, rank, local):
+    from rope_context_extension_sm_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    from rope_context_extension_sm_b200 import jetlong as jl
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L = PREFILL.seqlens[0]
+    # ---- inputs (host, seeded), then resident in HBM ----
+    q_h, k_h, v_h, cu_h = I.prefill_inputs(PREFILL)
+    q_h, k_h, v_h = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    q, k, v, cu = q_h.to(dev), k_h.to(dev), v_h.to(dev), cu_h.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((PREFILL.n_q_heads, L), dtype=torch.float32, device=dev)
+    cos, sin = jl.jl_rope_tables(L, PREFILL.head_dim, PREFILL.rope_base, device=dev)
+    dk_h, dv_h = _build_decode_cache(DECODE_L)
+    dk, dv = dk_h.to(dev), dv_h.to(dev)
+    dq_h = I.decode_queries(DECODE, 1)[0].contiguous().pin_memory()
+    dq = dq_h.to(dev)
+    dsl = torch.tensor([DECODE_L], dtype=torch.int32, device=dev)
+    dout = torch.empty_like(dq)
+    dlse = torch.empty((1, DECODE.n_q_heads), dtype=torch.float32, device=dev)
+    dws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, DECODE.n_q_heads, DECODE.head_dim, DECODE_L),
+                      dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill():
+        jl.jl_bifocal_prefill(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin, out=out, lse=lse)
+
+    def decode():
+        jl.jl_bifocal_decode(dq, dk, dv, dsl, DECODE_L, DECODE.w0, DECODE.w_pretrained, cos, sin, out=dout,
+                             lse=dlse, workspace=dws)
+
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    jl.jl_sync_status()
+
+    sampler = ClockSampler(local)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    _barrier(world)
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(K):
+        ev[s][0].record(stream)
+        prefill()
+        ev[s][1].record(stream)
+        decode()
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    _barrier(world)
+    clocks = sampler.stop()
+    jl.jl_sync_status()
+    total_ms = _max_over_ranks(t_start.elapsed_time(t_end), world)
+    pre_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    dec_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
+    pre_avg = _max_over_ranks(sum(pre_ms) / K, world)
+    dec_avg = _max_over_ranks(sum(dec_ms) / K, world)
+
+    flops = PREFILL.useful_flops()
+    value = world * flops * K / (total_ms * 1e-3) / 1e12  # whole job, prefill flops over the step time
+    prefill_tflops = flops / (pre_avg * 1e-3) / 1e12
+    burst, sustained, hbm, peak_kind = _peaks()
+    kv_bytes = 2 * DECODE_L * DECODE.n_kv_heads * DECODE.head_dim * 2
+    dec_gbs = kv_bytes / (dec_avg * 1e-3) / 1e9
+
+    # ---- plain comparators, same run ----
+    def plain_prefill():
+        jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse)
+
+    def plain_decode():
+        jl.jl_plain_decode(dq, dk, dv, dsl, DECODE_L, cos, sin, out=dout, lse=dlse, workspace=dws)
+
+    def _time(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    plain_pre_ms = _time(plain_prefill, max(1, min(K, 3)))
+    plain_dec_ms = _time(plain_decode, 50)
+    bif_dec_ms_loop = _time(decode, 50)
+
+    # ---- decode at the other cache lengths (rotating caches so each launch streams from HBM) ----
+    sweep = {}
+    for Ld in DECODE.cache_lens:
+        if Ld == DECODE_L:
+            sweep[str(Ld)] = {"us": bif_dec_ms_loop * 1e3, "plain_us": plain_dec_ms * 1e3}
+            continue
+        bytes_one = 2 * Ld * DECODE.n_kv_heads * DECODE.head_dim * 2
+        n_rot = max(1, int(math.ceil(2 * 126e6 / bytes_one)))
+        caches = [(dk[:, :Ld].contiguous(), dv[:, :Ld].contiguous()) for _ in range(n_rot)]
+        sl = torch.tensor([Ld], dtype=torch.int32, device=dev)
+        ws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, DECODE.n_q_heads, DECODE.head_dim, Ld),
+                         dtype=torch.uint8, device=dev)
+        it = [0]
+
+        def dstep(plain=False):
+            kk, vv = caches[it[0] % n_rot]
+            it[0] += 1
+            if plain:
+                jl.jl_plain_decode(dq, kk, vv, sl, Ld, cos, sin, out=dout, lse=dlse, workspace=ws)
+            else:
+                jl.jl_bifocal_decode(dq, kk, vv, sl, Ld, DECODE.w0, DECODE.w_pretrained, cos, sin, out=dout,
+                                     lse=dlse, workspace=ws)
+
+        sweep[str(Ld)] = {"us": _time(dstep, 50) * 1e3, "plain_us": _time(lambda: dstep(True), 50) * 1e3,
+                          "rotating_caches": n_rot}
+        del caches
+    for Ld, rec in sweep.items():
+        rec["overhead_vs_plain"] = rec["us"] / rec["plain_us"] - 1.0
+        rec["hbm_gbs"] = 2 * int(Ld) * DECODE.n_kv_heads * DECODE.head_dim * 2 / (rec["us"] * 1e-6) / 1e9
+    jl.jl_sync_status()
+
+    # ---- end to end through host buffers (H2D inputs, D2H outputs inside the timed region) ----
+    out_h = torch.empty_like(q_h).pin_memory()
+    lse_h = torch.empty((PREFILL.n_q_heads, L), dtype=torch.float32).pin_memory()
+    dout_h = torch.empty_like(dq_h).pin_memory()
+    e2e_steps = max(1, min(K, 3))
+    _barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        dq.copy_(dq_h, non_blocking=True)
+        prefill()
+        decode()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        dout_h.copy_(dout, non_blocking=True)
+    b.record(stream)
+    _barrier(world)
+    e2e_ms = _max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h))
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, dout_h))
+
+    res = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, outlier-scaled key channels)",
+        "config": _config(),
+        "prefill": {
+            "ms": round(pre_avg, 4),
+            "useful_tflops": round(prefill_tflops, 2),
+            "frac_of_bf16_peak_measured_sustained": round(prefill_tflops / sustained, 4),
+            "frac_of_bf16_peak_measured_burst": round(prefill_tflops / burst, 4),
+            "frac_of_bf16_nominal_2250": round(prefill_tflops / 2250.0, 4),
+            "plain_ms": round(plain_pre_ms, 4),
+            "plain_useful_tflops": round(flops / (plain_pre_ms * 1e-3) / 1e12, 2),
+            "bifocal_over_plain_time": round(pre_avg / plain_pre_ms, 4),
+        },
+        "decode": {
+            "us_per_token": round(dec_avg * 1e3, 2),
+            "cache_len": DECODE_L,
+            "hbm_gbs": round(dec_gbs, 1),
+            "frac_of_hbm_measured": round(dec_gbs / hbm, 4),
+            "frac_of_hbm_nominal_8000": round(dec_gbs / 8000.0, 4),
+            "plain_us_per_token": round(plain_dec_ms * 1e3, 2),
+            "overhead_vs_plain": round(bif_dec_ms_loop / plain_dec_ms - 1.0, 4),
+            "sweep": {k_: {kk: (round(vv, 3) if isinstance(vv, float) else vv) for kk, vv in r.items()}
+                      for k_, r in sweep.items()},
+        },
+        "roofline": {
+            "kernel": "jl_prefill_kernel<128,2>",
+            "bound": "tensor",
+            "achieved": round(prefill_tflops, 2),
+            "peak": sustained,
+            "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long loop)",
+            "unit": "TFLOP/s",
+            "frac": round(prefill_tflops / sustained, 4),
+            "traffic": _traffic("prefill", PREFILL_SRC),
+            "algorithmic_bytes_per_launch": int(sum(t.numel() * t.element_size() for t in (q, k, v, out, lse))),
+        },
+        "e2e": {
+            "value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
+            "unit": UNIT,
+            "ms_per_step": round(e2e_ms, 3),
+            "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+        },
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return res
+
+
+# ----------------------------------------------------- CPU oracle (baseline) ----
+
+def _oracle_sample_rows(n_rows, seed=7):
+    rng = np.random.default_rng(seed)
+    L = PREFILL.seqlens[0]
+    pos = rng.integers(L // 2, L, n_rows)
+    head = rng.integers(0, PREFILL.n_q_heads, n_rows)
+    return pos, head
+
+
+def cpu_baseline(seconds=15.0, inputs=None):
+    """The fp64 oracle as it stands, on a bounded sample of the prefill workload: rows drawn
+    uniformly from the second half of the 128K sequence, all query heads of KV head 0."""
+    from oracle import oracle as O
+    if inputs is None:
+        q_h, k_h, v_h, _ = I.prefill_inputs(PREFILL)
+    else:
+        q_h, k_h, v_h = inputs
+    L = PREFILL.seqlens[0]
+    qb, kb, vb = I.bf16_bits(q_h), I.bf16_bits(k_h), I.bf16_bits(v_h)
+    group = PREFILL.n_q_heads // PREFILL.n_kv_heads
+    rng = np.random.default_rng(7)
+    n = 8
+    done_rows, done_flops, spent = 0, 0.0, 0.0
+    while spent < seconds:
+        pos = rng.integers(L // 2, L, n)
+        head = rng.integers(0, group, n)  # KV head 0's query heads
+        t0 = time.perf_counter()
+        O.bifocal_rows(qb, kb, vb, L, pos, head, w0=PREFILL.w0, w_pretrained=PREFILL.w_pretrained,
+                       rope_base=PREFILL.rope_base)
+        spent += time.perf_counter() - t0
+        done_rows += n
+        done_flops += float(np.sum(4.0 * PREFILL.head_dim * (pos + 1)))
+        n = min(n * 2, 256)
+    return {
+        "value": done_flops / spent / 1e12,
+        "unit": UNIT,
+        "cores": O.num_threads(),
+        "kind": "oracle",
+        "sample": f"{done_rows} query rows of the L=131072 prefill (positions in [65536, 131072), KV head 0), "
+                  f"{spent:.1f} s; useful flops of those rows / time",
+        "full_layer_estimate_s": PREFILL.useful_flops() / (done_flops / spent),
+    }
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    from oracle import oracle as O
+    q_h, k_h, v_h, _ = I.prefill_inputs(PREFILL)
+    inputs = (q_h, k_h, v_h)
+    for _ in range(args.warmup):
+        cpu_baseline(seconds=0.5, inputs=inputs)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps)))
+    vals = [cpu_baseline(seconds=per_step, inputs=inputs) for _ in range(args.steps)]
+    v = statistics.mean(r["value"] for r in vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16, outlier-scaled key channels)",
+        "config": _config(),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle",
+                         "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, world, rank)
+        if res is not None:
+            print(json.dumps(res))
+        return
+    world, rank, local = _dist_setup(args.gpus)
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -79,15 +79,16 @@ def _compare_all_rows(jl, cfg, plain=False):
 
 @pytest.mark.parametrize("n,d,base", [(256, 64, 1e4), (131072, 128, 1e6)])
 def test_rope_tables_match_fp64_rounded_once(jl, n, d, base):
+    """fp32 tables = fp64 cos/sin rounded once.  The device's fp64 pow/sincos and the
+    host's agree to ~1e-11 rad at p ~ 1.3e5, so compare absolutely: within half an fp32
+    ulp at magnitude 1 (2^-25) plus that slack, and bit-equal for almost every entry."""
     cos, sin = _tables(jl, n, d, base)
     jl.jl_sync_status()
     rc, rs = O.rope_cos_sin(n, d, base)
     for got, ref in ((cos, rc), (sin, rs)):
-        g = got.cpu().numpy()
-        r32 = ref.astype(np.float32)
-        ulps = np.abs(g.view(np.int32).astype(np.int64) - r32.view(np.int32).astype(np.int64))
-        assert ulps.max() <= 1, f"table differs from fp64-rounded by {ulps.max()} ulp"
-        assert (ulps > 0).mean() < 1e-3
+        g = got.cpu().numpy().astype(np.float64)
+        assert np.abs(g - ref).max() <= 2.0 ** -25 + 1e-9
+        assert (g != ref.astype(np.float32)).mean() < 1e-3
 
 
 # ----------------------------------------------------------------- prefill ----
