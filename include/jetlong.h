@@ -151,6 +151,37 @@ jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cach
                           float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                           jl_stream_t stream);
 
+/*
+ * jl_bifocal_decode without a caller workspace.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory, for
+ * example an engine plugin that is handed only its input and output buffers,
+ * or a serving loop that forbids cudaMalloc once it is running.  It computes
+ * exactly what jl_bifocal_decode computes and takes the same arguments minus
+ * the workspace.  It allocates nothing: the split-K scratch is a file-scope
+ * device array of jl_bifocal_decode_noalloc_scratch_bytes() bytes (8 MiB) that
+ * every GPU loading the library holds until the process exits.
+ *  - Sizes whose scratch would exceed that maximum (B * n_split * Hq *
+ *    (head_dim + 2) * 4 bytes, see jl_bifocal_decode_workspace_size) return
+ *    JL_ERR_INVALID with a message; B = 1, Hq = 32, head_dim = 128 fits up to
+ *    max_seqlen = 131072.
+ *  - The first call on a device looks up the array's device address (the
+ *    device current at the call is the one used); make that first call before
+ *    any stream capture.
+ *  - All calls on a device share the one array, and it keeps whatever the last
+ *    call left there (nothing in it needs to start at zero).  Calls whose
+ *    executions overlap on the GPU -- on different streams, or from different
+ *    host threads -- race on it: order them on one stream or use
+ *    jl_bifocal_decode with separate workspaces.
+ */
+jl_status jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                    int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                                    int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                                    const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out,
+                                    float* lse, jl_stream_t stream);
+
+/* Bytes of the static scratch behind jl_bifocal_decode_noalloc (per device). */
+size_t jl_bifocal_decode_noalloc_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -326,3 +326,69 @@ jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cach
 }
 
 }  // extern "C"
+
+// ======================================== decode without caller workspace ==
+//
+// For callers that cannot allocate device memory (see jl_bifocal_decode_noalloc
+// in jetlong.h).  The split-K partials live in one file-scope device array that
+// every GPU loading this library holds until the process exits.  Host code may
+// not pass the array's name to a kernel (on the host it is only a stand-in), so
+// the device address is looked up once per device with cudaGetSymbolAddress
+// while that device is current, then cached.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+jl_status static_scratch_for_current_device(void** addr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(JL_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return JL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t jl_bifocal_decode_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
+
+jl_status jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                    int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
+                                    int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                                    const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out,
+                                    float* lse, jl_stream_t stream) {
+  const size_t need = decode_ws_bytes(B, Hq, head_dim, max_seqlen);
+  if (need > kStaticScratchBytes)
+    return fail(JL_ERR_INVALID,
+                "jl_bifocal_decode_noalloc: B=%d, Hq=%d, head_dim=%d, max_seqlen=%d need %zu bytes of scratch, "
+                "more than the %zu-byte static scratch; use jl_bifocal_decode with a caller workspace",
+                B, Hq, head_dim, max_seqlen, need, kStaticScratchBytes);
+  if (B <= 0) return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim,
+                                   w0, w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse,
+                                   nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+  void* scratch = nullptr;
+  const jl_status s = static_scratch_for_current_device(&scratch);
+  if (s != JL_OK) return s;
+  // Every partial the combine step reads is written earlier in the same call, so
+  // nothing in the scratch needs clearing between calls.
+  return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim, w0,
+                       w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, scratch,
+                       kStaticScratchBytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

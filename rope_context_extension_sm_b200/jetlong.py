@@ -45,6 +45,9 @@ SIGNATURES = {
     "jl_bifocal_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "jl_plain_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
                                        _f32, _vp, _vp, _vp, _sz, _vp]),
+    "jl_bifocal_decode_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
+                                                 _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
+    "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -205,6 +208,29 @@ def jl_plain_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, cos, sin, *, 
                                 max_seqlen, hq, hkv, d, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale,
                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "jl_plain_decode")
+    return out, lse
+
+
+def jl_bifocal_decode_noalloc_scratch_bytes() -> int:
+    return int(_lib.jl_bifocal_decode_noalloc_scratch_bytes())
+
+
+def jl_bifocal_decode_noalloc(q, k_cache, v_cache, seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin,
+                              *, out, lse=None, softmax_scale: float = 0.0, stream=None):
+    """jl_bifocal_decode for callers that cannot allocate: the library uses its own
+    static per-device scratch, so the caller passes only inputs and outputs (out and
+    lse are caller-owned; lse may be None).  Calls that overlap on the GPU race on
+    the shared scratch."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(seqlens, torch.int32, "seqlens", 1)
+    _need(out, torch.bfloat16, "out", 3)
+    B, hq, d = q.shape
+    _check(_lib.jl_bifocal_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, k_cache.shape[1],
+                                          max_seqlen, hq, k_cache.shape[2], d, w0, w_pretrained, _ptr(cos),
+                                          _ptr(sin), cos.shape[0], softmax_scale, _ptr(out), _ptr(lse),
+                                          _stream(stream)), "jl_bifocal_decode_noalloc")
     return out, lse
 
 
