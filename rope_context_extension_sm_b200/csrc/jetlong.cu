@@ -160,7 +160,7 @@ jl_status launch_decode(const jl::DecodeParams& prm, int B, cudaStream_t st) {
   jl::jl_decode_split_kernel<D, GROUP, PLAIN><<<grid, jl::kDecodeThreads, 0, st>>>(prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  jl::jl_decode_combine_kernel<D><<<dim3(prm.Hq, B), D, 0, st>>>(prm);
+  jl::jl_decode_combine_kernel<D><<<dim3(prm.Hq, B), jl::kCombineThreads, 0, st>>>(prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return ok();

@@ -258,40 +258,64 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
   }
 }
 
-// Merge the per-split partials of one (batch entry, query head).
+// Merge the per-split partials of one (batch entry, query head).  Eight warps
+// walk the splits in parallel (lane owns D/32 channels), each keeping an online
+// (max, sum, o) state; the warps' states are merged in shared memory.
+constexpr int kCombineThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(D) jl_decode_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kCombineThreads) jl_decode_combine_kernel(const DecodeParams p) {
+  constexpr int CPL = D / 32;  // channels per lane
+  constexpr int NW = kCombineThreads / 32;
   const int qh = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = p.seqlens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
   const float* base = p.ws + (static_cast<int64_t>(b) * p.n_split * p.Hq + qh) * (D + 2);
   const int64_t sstride = static_cast<int64_t>(p.Hq) * (D + 2);
-  __shared__ float red[D / 32];
-  __shared__ float mshared;
-  float mx = -INFINITY;
-  for (int s = threadIdx.x; s < ns; s += D) mx = fmaxf(mx, base[s * sstride]);
+  __shared__ float sm_m[NW], sm_l[NW];
+  __shared__ float sm_o[NW][D];
+  float m = -INFINITY, l = 0.f, acc[CPL];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float v = red[0];
-    for (int w = 1; w < D / 32; ++w) v = fmaxf(v, red[w]);
-    mshared = v;
-  }
-  __syncthreads();
-  const float M = mshared;
-  float acc = 0.f, lsum = 0.f;
-  for (int s = 0; s < ns; ++s) {
+  for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < ns; s += NW) {
     const float* ps = base + s * sstride;
-    const float ms = ps[0];
-    const float sc = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
-    acc = fmaf(ps[2 + threadIdx.x], sc, acc);
-    lsum = fmaf(ps[1], sc, lsum);
+    const float ms = ps[0], ls = ps[1];
+    float o[CPL];
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) o[e] = ps[2 + lane * CPL + e];
+    if (ms == -INFINITY) continue;
+    const float mn = fmaxf(m, ms);
+    const float a = (m == -INFINITY) ? 0.f : ex2_approx(m - mn);
+    const float bb = ex2_approx(ms - mn);
+    l = l * a + ls * bb;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] = acc[e] * a + o[e] * bb;
+    m = mn;
   }
-  p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + threadIdx.x] = __float2bfloat16_rn(acc / lsum);
-  if (threadIdx.x == 0 && p.lse != nullptr)
-    p.lse[static_cast<int64_t>(b) * p.Hq + qh] = (M + log2f(lsum)) * 0.69314718055994531f;
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) sm_o[warp][lane * CPL + e] = acc[e];
+  if (lane == 0) {
+    sm_m[warp] = m;
+    sm_l[warp] = l;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += kCombineThreads) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w]);
+    float o = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float sc = (sm_m[w] == -INFINITY) ? 0.f : ex2_approx(sm_m[w] - M);
+      o = fmaf(sm_o[w][c], sc, o);
+      lsum = fmaf(sm_l[w], sc, lsum);
+    }
+    p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(o / lsum);
+    if (c == 0 && p.lse != nullptr)
+      p.lse[static_cast<int64_t>(b) * p.Hq + qh] = (M + log2f(lsum)) * 0.69314718055994531f;
+  }
 }
 
 }  // namespace jl

@@ -23,10 +23,13 @@
 // KV head (GQA).  Each K/V tile is loaded once by TMA and feeds all NQT heads.
 //   warp 0      TMA producer (Q, K, V tiles; 128B-swizzled boxes)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-3   in-place RoPE rotation of the Q and K tiles in shared memory
-//               (base rows R(x) or remote rows R(f(x)), from the fp32 tables)
 //   warps 4..   one warpgroup per query head: softmax on S read from TMEM,
 //               P written back to TMEM (bf16), O rescale, epilogue
+//   4 more      in-place RoPE rotation of the Q and K tiles in shared memory
+//   warps       (base rows R(x) or remote rows R(f(x))); each owns 32 rows and
+//               steps its cos/sin factors along the rows by complex
+//               multiplication with e^{i theta_c}, anchored once per tile on a
+//               table row prefetched a tile ahead (no table load per row)
 // TMEM columns: S_t at 128 t, O_t at 128 NQT + D t; P_t aliases S_t.
 // With NQT = 2 the MMA issue order S0(n), PV1(n-1), S1(n), PV0(n) lets one
 // head's softmax overlap the other head's tensor-core work.
@@ -72,7 +75,12 @@ struct PrefillLayout {
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
   static constexpr int kColsUsed = NQT * 128 + NQT * D;
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
-  static constexpr int kThreads = 128 + NQT * 128;
+  static constexpr int kRotWarps = 4;
+  static constexpr int kThreads = 32 * (2 + kRotWarps) + NQT * 128;
+  // warps: 0 producer, 1 MMA, 2-3 rotation, 4 .. 4+4NQT-1 softmax, then 2 more rotation warps
+  __device__ static int rot_index(int warp) {
+    return warp < 4 ? warp - 2 : (warp >= 4 + 4 * NQT ? warp - (4 + 4 * NQT) + 2 : -1);
+  }
 };
 
 struct PrefillBars {
@@ -118,53 +126,91 @@ struct TileSchedule {
   }
 };
 
-// Rotate one 128-byte-swizzled row of a [128 rows][D] bf16 tile in place by R(p).
-// Lane l owns frequency pairs c in [l*FPL, l*FPL + FPL) with partners c + D/2.
+// cos/sin of the frequencies a lane owns: c = 2l, 2l+1 (D = 128) or c = l (D = 64);
+// each is paired with channel c + D/2 (rotate-half).
 template <int D>
-__device__ __forceinline__ void rotate_row_inplace(uint8_t* tile, int r, const float* __restrict__ cos_row,
-                                                   const float* __restrict__ sin_row, int lane) {
+struct RotFactor {
+  static constexpr int NF = D / 64;
+  float c[NF], s[NF];
+};
+
+template <int D>
+__device__ __forceinline__ void load_factor(RotFactor<D>& f, const PrefillParams& p, int64_t row, int lane) {
+  const int64_t max_row = p.n_tab_rows - 1;
+  row = row > max_row ? max_row : row;  // only rows past every sequence end are clamped
   if constexpr (D == 128) {
-    // elements 2l, 2l+1 (box 0) and 64+2l, 64+2l+1 (box 1), same swizzled offset
-    const int off = r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + ((lane & 3) << 2);
+    const float2 cc = __ldg(reinterpret_cast<const float2*>(p.cos_tab + row * 64 + 2 * lane));
+    const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + row * 64 + 2 * lane));
+    f.c[0] = cc.x; f.c[1] = cc.y; f.s[0] = ss.x; f.s[1] = ss.y;
+  } else {
+    f.c[0] = __ldg(p.cos_tab + row * 32 + lane);
+    f.s[0] = __ldg(p.sin_tab + row * 32 + lane);
+  }
+}
+
+// f <- f * e^{i theta}: R(m) -> R(m + 1).
+template <int D>
+__device__ __forceinline__ void advance(RotFactor<D>& f, const RotFactor<D>& st) {
+#pragma unroll
+  for (int i = 0; i < RotFactor<D>::NF; ++i) {
+    const float c = f.c[i] * st.c[i] - f.s[i] * st.s[i];
+    const float sn = f.s[i] * st.c[i] + f.c[i] * st.s[i];
+    f.c[i] = c;
+    f.s[i] = sn;
+  }
+}
+
+// Rotate row r of a 128-byte-swizzled [128 rows][D] bf16 tile in place with factor f.
+template <int D>
+__device__ __forceinline__ void rotate_row(uint8_t* tile, int r, const RotFactor<D>& f, int lane) {
+  if constexpr (D == 128) {
+    // elements 2l, 2l+1 (box 0) and 64+2l, 64+2l+1 (box 1) share the swizzled offset
+    const int off = r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + ((lane & 3) << 2);
     __nv_bfloat162* plo = reinterpret_cast<__nv_bfloat162*>(tile + off);
     __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
-    const float2 cs = *reinterpret_cast<const float2*>(cos_row + 2 * lane);
-    const float2 sn = *reinterpret_cast<const float2*>(sin_row + 2 * lane);
     const float2 a = __bfloat1622float2(*plo);
     const float2 b = __bfloat1622float2(*phi);
     float2 ya, yb;
-    ya.x = a.x * cs.x - b.x * sn.x;
-    yb.x = b.x * cs.x + a.x * sn.x;
-    ya.y = a.y * cs.y - b.y * sn.y;
-    yb.y = b.y * cs.y + a.y * sn.y;
+    ya.x = a.x * f.c[0] - b.x * f.s[0];
+    yb.x = b.x * f.c[0] + a.x * f.s[0];
+    ya.y = a.y * f.c[1] - b.y * f.s[1];
+    yb.y = b.y * f.c[1] + a.y * f.s[1];
     *plo = __float22bfloat162_rn(ya);
     *phi = __float22bfloat162_rn(yb);
   } else {
-    // D == 64: element l and l + 32 of the single box
+    // D == 64: elements l and l + 32 of the single box
     const int c0 = lane, c1 = lane + 32;
     const int off0 = r * 128 + ((((c0 * 2) >> 4) ^ (r & 7)) << 4) + ((c0 * 2) & 15);
     const int off1 = r * 128 + ((((c1 * 2) >> 4) ^ (r & 7)) << 4) + ((c1 * 2) & 15);
     __nv_bfloat16* pa = reinterpret_cast<__nv_bfloat16*>(tile + off0);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(tile + off1);
-    const float cs = cos_row[lane], sn = sin_row[lane];
     const float a = __bfloat162float(*pa), b = __bfloat162float(*pb);
-    *pa = __float2bfloat16_rn(a * cs - b * sn);
-    *pb = __float2bfloat16_rn(b * cs + a * sn);
+    *pa = __float2bfloat16_rn(a * f.c[0] - b * f.s[0]);
+    *pb = __float2bfloat16_rn(b * f.c[0] + a * f.s[0]);
   }
 }
 
-// Rotate rows r = r0, r0 + stride, ... of a tile whose row r sits at position base + r.
+// Table row of the first row of rotation slice rw: position base + 32 rw, or its
+// remote position floor(./G) (g = 1 selects base positions).
+__device__ __forceinline__ int64_t slice_anchor_row(int base, int rw, int g) {
+  const int pos = base + 32 * rw;
+  return g == 1 ? pos : pos / g;
+}
+
+// Rotate rows [32 rw, 32 rw + 32) of a tile whose row r sits at position base + r:
+// by R(pos) when g == 1, by R(floor(pos / g)) otherwise.  f is the factor of the
+// slice's first row; the remote position advances by one every g rows.
 template <int D>
-__device__ __forceinline__ void rotate_tile(uint8_t* tile, int r0, int stride, int base, bool remote, int G,
-                                            const PrefillParams& p, int lane) {
-  constexpr int HALF = D / 2;
-  const int64_t max_row = p.n_tab_rows - 1;
+__device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, int g, RotFactor<D> f,
+                                             const RotFactor<D>& st, int lane) {
+  int cnt = (base + 32 * rw) % g;
 #pragma unroll 4
-  for (int r = r0; r < kBM; r += stride) {
-    int pos = base + r;
-    int64_t row = remote ? (pos / G) : pos;
-    row = row > max_row ? max_row : row;  // rows past the sequence end are masked later
-    rotate_row_inplace<D>(tile, r, p.cos_tab + row * HALF, p.sin_tab + row * HALF, lane);
+  for (int r = 0; r < 32; ++r) {
+    rotate_row<D>(tile, 32 * rw + r, f, lane);
+    if (++cnt == g) {
+      cnt = 0;
+      advance<D>(f, st);
+    }
   }
 }
 
@@ -212,11 +258,11 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_ready, 2);
+    mbar_init(&bars->q_ready, Lay::kRotWarps);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_ready[s], 2);
+      mbar_init(&bars->k_ready[s], Lay::kRotWarps);
       mbar_init(&bars->k_empty[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
@@ -352,22 +398,33 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       umma_commit(&bars->teardown);
       mbar_wait_bounded(&bars->teardown, 0);
     }
-  } else if (warp < 4) {
+  } else if (Lay::rot_index(warp) >= 0) {
     // ------------------------------------------------------------ rotation
-    const int rw = warp - 2;
+    const int rw = Lay::rot_index(warp);
+    RotFactor<D> step;  // e^{i theta_c}: table row 1
+    load_factor<D>(step, p, 1, lane);
+    auto key_anchor = [&](int n) {
+      return slice_anchor_row(sc.kt(n) * kBN, rw, sc.remote(n) ? G : 1);
+    };
+    RotFactor<D> fk_next;
+    load_factor<D>(fk_next, p, key_anchor(0), lane);
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
+      const int g = remote ? G : 1;
       if (n == 0 || n == sc.R) {
+        RotFactor<D> fq;
+        load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane);
         if (!mbar_wait(&bars->q_full, n == 0 ? 0 : 1, abort)) break;
-        for (int t = 0; t < NQT; ++t)
-          rotate_tile<D>(sQ + t * Lay::kTileBytes, rw, 2, sc.q_lo, remote, G, p, lane);
+        for (int t = 0; t < NQT; ++t) rotate_slice<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, step, lane);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_ready);
       }
+      const RotFactor<D> fk = fk_next;
+      if (n + 1 < sc.n_virt) load_factor<D>(fk_next, p, key_anchor(n + 1), lane);  // prefetch a tile ahead
       const int s = n % kStages;
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
-      rotate_tile<D>(sK + s * Lay::kTileBytes, rw, 2, sc.kt(n) * kBN, remote, G, p, lane);
+      rotate_slice<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);
@@ -388,7 +445,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     for (int n = 0; n < sc.n_virt; ++n) {
       if (!(ok = mbar_wait(&bars->s_full[t], n & 1, abort))) break;
       tc_fence_after();
-      // Pass A: row max over the (masked) scores, 32 columns at a time.
+      // Pass A: row max over the (masked) scores, 64 columns at a time.
       const bool msk = sc.masked(n);
       const int hi = i - sc.kt(n) * kBN;  // causal: keep column c <= hi
       const int edge = hi - sc.w0;        // remote keeps c <= edge, local keeps c > edge
@@ -397,14 +454,23 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const int keep_hi = msk ? (rem ? edge : hi) : kBN;    // keep c <= keep_hi
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + c * 32, sr);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sr[64];
+        tmem_ld64(t_s + c * 64, sr);
+        if (msk) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = c * 32 + e;
-          const float x = __uint_as_float(sr[e]);
-          mx = (col > keep_lo && col <= keep_hi) ? fmaxf(mx, x) : mx;
+          for (int e = 0; e < 64; ++e) {
+            const int col = c * 64 + e;
+            mx = (col > keep_lo && col <= keep_hi) ? fmaxf(mx, __uint_as_float(sr[e])) : mx;
+          }
+        } else {
+          float m2 = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            mx = fmaxf(mx, __uint_as_float(sr[e]));
+            m2 = fmaxf(m2, __uint_as_float(sr[e + 1]));
+          }
+          mx = fmaxf(mx, m2);
         }
       }
       const float m_new = fmaxf(m_run, mx * sl2);
@@ -414,32 +480,31 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (resc || m_run == -INFINITY) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       // Pass B: P = 2^(s * scale_log2 - m), written back over S as bf16 pairs.
-      // Chunk c reads S columns [32c, 32c+32) and writes P columns [16c, 16c+16);
+      // Chunk c reads S columns [64c, 64c+64) and writes P columns [32c, 32c+32);
       // every write lands on S columns that were already read.
-      float lsum = 0.f;
+      float lsum = 0.f, lsum2 = 0.f;
+      const float neg_m = -m_use;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + c * 32, sr);
-        uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sr[64];
+        tmem_ld64(t_s + c * 64, sr);
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c * 32 + 2 * e;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, -m_use));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, -m_use));
-          p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
-          p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
-          lsum += p0 + p1;
+        for (int e = 0; e < 32; ++e) {
+          const int col = c * 64 + 2 * e;
+          float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m));
+          if (msk) {
+            p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
+            p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
+          }
+          lsum += p0;
+          lsum2 += p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
-        // 16 packed words = keys 32c .. 32c+31 -> columns 128 t + 16 c .. + 15 (P_t aliases S_t)
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-            "%14, %15, %16};\n" ::"r"(t_s + c * 16),
-            "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7]),
-            "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-            : "memory");
+        tmem_st32(t_s + c * 32, pk);
       }
+      lsum += lsum2;
       l_run = l_run * alpha + lsum;
       // O_t *= alpha for the rows whose max moved (PV_t(n-1) is complete: it was
       // issued before S_t(n), whose commit we waited on).
