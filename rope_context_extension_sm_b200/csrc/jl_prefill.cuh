@@ -204,13 +204,35 @@ template <int D>
 __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, int g, RotFactor<D> f,
                                              const RotFactor<D>& st, int lane) {
   int cnt = (base + 32 * rw) % g;
+  uint8_t* slice = tile + 32 * rw * 128;  // 32 rows x 128 B; row & 7 == r & 7
 #pragma unroll 4
   for (int r = 0; r < 32; ++r) {
-    rotate_row<D>(tile, 32 * rw + r, f, lane);
+    rotate_row<D>(slice, r, f, lane);
     if (++cnt == g) {
       cnt = 0;
       advance<D>(f, st);
     }
+  }
+}
+
+// Softmax pass B on one 64-column chunk: p = 2^(s * sl2 - m) (zero outside
+// [keep_lo + 1, keep_hi] when MASK), packed to bf16 pairs; returns the two
+// partial row sums.  Straight-line code: no branch inside the chunk.
+template <bool MASK>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[64], uint32_t (&pk)[32], int col0, float sl2,
+                                              float neg_m, int keep_lo, int keep_hi, float& lsum, float& lsum2) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m));
+    float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m));
+    if constexpr (MASK) {
+      const int col = col0 + 2 * e;
+      p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
+      p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
+    }
+    lsum += p0;
+    lsum2 += p1;
+    pk[e] = pack_bf16x2(p0, p1);
   }
 }
 
@@ -466,9 +488,9 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         } else {
           float m2 = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            mx = fmaxf(mx, __uint_as_float(sr[e]));
-            m2 = fmaxf(m2, __uint_as_float(sr[e + 1]));
+          for (int e = 0; e < 64; e += 4) {
+            mx = fmax3(mx, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            m2 = fmax3(m2, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
           }
           mx = fmaxf(mx, m2);
         }
@@ -484,25 +506,22 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       // every write lands on S columns that were already read.
       float lsum = 0.f, lsum2 = 0.f;
       const float neg_m = -m_use;
+      if (msk) {
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sr[64];
-        tmem_ld64(t_s + c * 64, sr);
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = c * 64 + 2 * e;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m));
-          if (msk) {
-            p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
-            p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
-          }
-          lsum += p0;
-          lsum2 += p1;
-          pk[e] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sr[64], pk[32];
+          tmem_ld64(t_s + c * 64, sr);
+          softmax_chunk<true>(sr, pk, c * 64, sl2, neg_m, keep_lo, keep_hi, lsum, lsum2);
+          tmem_st32(t_s + c * 32, pk);
         }
-        tmem_st32(t_s + c * 32, pk);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sr[64], pk[32];
+          tmem_ld64(t_s + c * 64, sr);
+          softmax_chunk<false>(sr, pk, c * 64, sl2, neg_m, keep_lo, keep_hi, lsum, lsum2);
+          tmem_st32(t_s + c * 32, pk);
+        }
       }
       lsum += lsum2;
       l_run = l_run * alpha + lsum;
