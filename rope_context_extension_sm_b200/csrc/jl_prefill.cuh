@@ -248,12 +248,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, false, true);
 
-  // ---- work item (heaviest query blocks first) ----
-  const int per = p.batch * p.Hkv * p.slots;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x) / per;
-  const int rem = static_cast<int>(blockIdx.x) % per;
-  const int b = rem / (p.Hkv * p.slots);
-  const int hkv = (rem / p.slots) % p.Hkv;
+  // ---- work item: KV-head-major so the CTAs in flight share one head's K/V in
+  // L2; within a head, heaviest query blocks first ----
+  const int per_head = p.n_qtiles * p.batch * p.slots;
+  const int hkv = static_cast<int>(blockIdx.x) / per_head;
+  const int rem = static_cast<int>(blockIdx.x) % per_head;
+  const int qt = p.n_qtiles - 1 - rem / (p.batch * p.slots);
+  const int b = (rem / p.slots) % p.batch;
   const int slot = rem % p.slots;
   const int h0 = hkv * p.group + slot * NQT;
   const int seq0 = p.cu_seqlens[b];
