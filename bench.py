@@ -91,7 +91,7 @@ DECODE_SRC = ["rope_context_extension_sm_b200/csrc/jl_decode.cuh", "rope_context
 def _traffic(kernel, files):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
     try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
             rec = json.load(f).get(kernel)
     except (OSError, ValueError):
         return None
