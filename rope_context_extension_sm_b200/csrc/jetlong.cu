@@ -14,6 +14,7 @@
 
 #include "jetlong.h"
 #include "jl_decode.cuh"
+#include "jl_decode_tc.cuh"
 #include "jl_prefill.cuh"
 #include "jl_tables.cuh"
 
@@ -148,10 +149,52 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
 
 // ------------------------------------------------------------------ decode --
 
-int decode_chunk(int32_t max_seqlen) {
+// Tensor-core decode (head_dim 128, up to 16 query heads per KV head) splits the
+// keys in chunks of whole 128-key tiles, sized for about four waves of CTAs; the
+// other shapes use the CUDA-core split kernel.
+bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) { return head_dim == 128 && Hq / Hkv <= 16; }
+
+// Keys per split.  CUDA-core kernel: a power of two in [64, 512].  Tensor-core
+// kernel: whole 128-key tiles, sized so that 8 KV heads x B entries give about
+// four waves of CTAs (the split count depends only on B and max_seqlen, never on
+// the head counts, so the workspace-size query below can bound it).
+int chunk_cuda_core(int32_t max_seqlen) {
   int c = 64;
   while (c < 512 && static_cast<int64_t>(c) * 256 < max_seqlen) c *= 2;
   return c;
+}
+
+int chunk_tc(int32_t B, int32_t max_seqlen) {
+  const int64_t tiles = (static_cast<int64_t>(max_seqlen) + jl::kDecTile - 1) / jl::kDecTile;
+  const int64_t want_ctas = 148 * 4;
+  int64_t per = (tiles * 8 * B + want_ctas - 1) / want_ctas;
+  per = per < 1 ? 1 : per;
+  return static_cast<int>(per * jl::kDecTile);
+}
+
+template <int GROUP, bool PLAIN>
+jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) {
+  using Lay = jl::DecTcLayout;
+  CUtensorMap tk, tv;
+  jl_status s;
+  const int64_t rows = static_cast<int64_t>(B) * prm.cache_stride;
+  if ((s = make_map(&tk, prm.k, rows, prm.Hkv, 128)) != JL_OK) return s;
+  if ((s = make_map(&tv, prm.v, rows, prm.Hkv, 128)) != JL_OK) return s;
+  auto kern = jl::jl_decode_tc_kernel<GROUP, PLAIN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
+  dim3 grid(prm.Hkv, prm.n_split, B);
+  kern<<<grid, Lay::kThreads, Lay::kAlloc, st>>>(tk, tv, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  jl::jl_decode_combine_kernel<128><<<dim3(prm.Hq, B), jl::kCombineThreads, 0, st>>>(prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return ok();
 }
 
 template <int D, int GROUP, bool PLAIN>
@@ -168,20 +211,39 @@ jl_status launch_decode(const jl::DecodeParams& prm, int B, cudaStream_t st) {
 
 template <int D, bool PLAIN>
 jl_status dispatch_group(const jl::DecodeParams& prm, int B, cudaStream_t st) {
+  if (decode_uses_tc(D, prm.Hq, prm.Hkv)) {
+    switch (prm.group) {
+      case 1: return launch_decode_tc<1, PLAIN>(prm, B, st);
+      case 2: return launch_decode_tc<2, PLAIN>(prm, B, st);
+      case 4: return launch_decode_tc<4, PLAIN>(prm, B, st);
+      case 8: return launch_decode_tc<8, PLAIN>(prm, B, st);
+      case 16: return launch_decode_tc<16, PLAIN>(prm, B, st);
+      default: break;
+    }
+  }
   switch (prm.group) {
     case 1: return launch_decode<D, 1, PLAIN>(prm, B, st);
     case 2: return launch_decode<D, 2, PLAIN>(prm, B, st);
     case 4: return launch_decode<D, 4, PLAIN>(prm, B, st);
     case 8: return launch_decode<D, 8, PLAIN>(prm, B, st);
-    default: return fail(JL_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8} (got %d)", prm.group);
+    default: return fail(JL_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8, 16} (got %d)", prm.group);
   }
 }
 
-size_t decode_ws_bytes(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {
-  if (B <= 0 || Hq <= 0 || head_dim <= 0 || max_seqlen <= 0) return 0;
-  const int chunk = decode_chunk(max_seqlen);
+size_t ws_bytes_for(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen, int chunk) {
   const int64_t n_split = (max_seqlen + chunk - 1) / chunk;
   return static_cast<size_t>(B) * n_split * Hq * (head_dim + 2) * sizeof(float);
+}
+
+// Upper bound over both decode kernels (the query does not know Hkv, which picks the kernel).
+size_t decode_ws_bytes(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {
+  if (B <= 0 || Hq <= 0 || head_dim <= 0 || max_seqlen <= 0) return 0;
+  size_t n = ws_bytes_for(B, Hq, head_dim, max_seqlen, chunk_cuda_core(max_seqlen));
+  if (head_dim == 128) {
+    const size_t t = ws_bytes_for(B, Hq, head_dim, max_seqlen, chunk_tc(B, max_seqlen));
+    n = t > n ? t : n;
+  }
+  return n;
 }
 
 jl_status decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, int32_t B,
@@ -203,6 +265,8 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
                 max_seqlen);
   if (n_tab_rows < max_seqlen)
     return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_seqlen (%d)", (long long)n_tab_rows, max_seqlen);
+  if (static_cast<int64_t>(B) * cache_stride > 0x7fffffffLL)
+    return fail(JL_ERR_UNSUPPORTED, "B * cache_stride must be < 2^31 (got %lld)", (long long)B * cache_stride);
   if (!q || !k_cache || !v_cache || !seqlens || !cos_tab || !sin_tab || !out || !workspace)
     return fail(JL_ERR_INVALID, "null pointer argument");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace) ||
@@ -222,13 +286,14 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
   prm.cache_stride = cache_stride;
+  prm.n_tab_rows = n_tab_rows;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
   prm.w0 = w0;
   prm.w_pre = w_pretrained;
   prm.plain = plain;
-  prm.chunk = decode_chunk(max_seqlen);
+  prm.chunk = decode_uses_tc(head_dim, Hq, Hkv) ? chunk_tc(B, max_seqlen) : chunk_cuda_core(max_seqlen);
   prm.n_split = (max_seqlen + prm.chunk - 1) / prm.chunk;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   prm.scale_log2 = scale * 1.4426950408889634f;

@@ -37,6 +37,7 @@ struct DecodeParams {
   __nv_bfloat16* out;
   float* lse;
   int64_t cache_stride;   // positions per batch entry
+  int64_t n_tab_rows;     // rows of cos_tab / sin_tab
   int32_t Hq, Hkv, group;
   int32_t w0, w_pre, plain;
   int32_t chunk, n_split;
@@ -258,9 +259,10 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
   }
 }
 
-// Merge the per-split partials of one (batch entry, query head).  Eight warps
-// walk the splits in parallel (lane owns D/32 channels), each keeping an online
-// (max, sum, o) state; the warps' states are merged in shared memory.
+// Merge the per-split partials of one (batch entry, query head).  Phase 1: the
+// block's maximum over the split maxima.  Phase 2: eight warps walk the splits
+// (lane owns D/32 channels) with every load independent of the previous one;
+// the warps' sums are added in shared memory.
 constexpr int kCombineThreads = 256;
 
 template <int D>
@@ -273,45 +275,40 @@ __global__ void __launch_bounds__(kCombineThreads) jl_decode_combine_kernel(cons
   const int ns = (L + p.chunk - 1) / p.chunk;
   const float* base = p.ws + (static_cast<int64_t>(b) * p.n_split * p.Hq + qh) * (D + 2);
   const int64_t sstride = static_cast<int64_t>(p.Hq) * (D + 2);
-  __shared__ float sm_m[NW], sm_l[NW];
+  __shared__ float sm_red[NW], sm_l[NW];
   __shared__ float sm_o[NW][D];
-  float m = -INFINITY, l = 0.f, acc[CPL];
+  float mx = -INFINITY;
+  for (int s = threadIdx.x; s < ns; s += kCombineThreads) mx = fmaxf(mx, base[s * sstride]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) sm_red[warp] = mx;
+  __syncthreads();
+  float M = sm_red[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, sm_red[w]);
+  float l = 0.f, acc[CPL];
 #pragma unroll
   for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
 #pragma unroll 4
   for (int s = warp; s < ns; s += NW) {
     const float* ps = base + s * sstride;
-    const float ms = ps[0], ls = ps[1];
-    float o[CPL];
+    const float ms = ps[0];
+    const float sc = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
+    l = fmaf(ps[1], sc, l);
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) o[e] = ps[2 + lane * CPL + e];
-    if (ms == -INFINITY) continue;
-    const float mn = fmaxf(m, ms);
-    const float a = (m == -INFINITY) ? 0.f : ex2_approx(m - mn);
-    const float bb = ex2_approx(ms - mn);
-    l = l * a + ls * bb;
-#pragma unroll
-    for (int e = 0; e < CPL; ++e) acc[e] = acc[e] * a + o[e] * bb;
-    m = mn;
+    for (int e = 0; e < CPL; ++e) acc[e] = fmaf(ps[2 + lane * CPL + e], sc, acc[e]);
   }
 #pragma unroll
   for (int e = 0; e < CPL; ++e) sm_o[warp][lane * CPL + e] = acc[e];
-  if (lane == 0) {
-    sm_m[warp] = m;
-    sm_l[warp] = l;
-  }
+  if (lane == 0) sm_l[warp] = l;
   __syncthreads();
+  float lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) lsum += sm_l[w];
   for (int c = threadIdx.x; c < D; c += kCombineThreads) {
-    float M = -INFINITY;
+    float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w]);
-    float o = 0.f, lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float sc = (sm_m[w] == -INFINITY) ? 0.f : ex2_approx(sm_m[w] - M);
-      o = fmaf(sm_o[w][c], sc, o);
-      lsum = fmaf(sm_l[w], sc, lsum);
-    }
+    for (int w = 0; w < NW; ++w) o += sm_o[w][c];
     p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(o / lsum);
     if (c == 0 && p.lse != nullptr)
       p.lse[static_cast<int64_t>(b) * p.Hq + qh] = (M + log2f(lsum)) * 0.69314718055994531f;

@@ -1,0 +1,434 @@
+// jl_decode_tc.cuh -- split-K bifocal decode on sm_100a with the keys on the
+// tensor-core M dimension (head_dim 128, up to 16 query heads per KV head).
+//
+// Method: "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
+// RoPE", Methodology section 2, on-the-fly correction rotation.  The cache holds
+// base keys k~_j = R(j) k_j and is only read.  Remote keys (i - j >= w0) score
+// <R(f(i) - i) q~, R(f(j) - j) k~_j> = <R(f(i)) q, R(f(j)) k_j>; local keys score
+// <q~, k~_j>.
+//
+// CTA = (KV head, chunk of keys, batch entry).  Per 128-key tile:
+//   warp 0      TMA producer: raw K and V tiles (3 stages)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-3,  correction warps: rotate the remote rows of the K tile in place
+//   8-13        by R(-(j - f(j))) (cos/sin stepped along the rows by complex
+//               multiplication, anchored on a table row prefetched a tile ahead)
+//   warps 4-7   softmax, thread = key row of S^T and channel row of O^T
+// MMAs:  S^T[128 keys x 32] = K_tile . [R(f(i)-i) q~ (16 rows) | q~ (16 rows)]^T
+//        O^T[128 ch x 16]  += V_tile^T . P^T          (A = V tile, MN-major)
+// Each key row picks the remote or the local half of its S^T row, so the tile
+// that straddles the window edge needs no second visit.  Per-head maxima are
+// reduced across the 128 threads each tile; row sums stay per thread and are
+// reduced once at the end.  The partial (m, l, o) per query head goes to the
+// workspace; jl_decode_combine_kernel merges the splits.
+#pragma once
+
+#include "jl_decode.cuh"
+#include "jl_device.cuh"
+
+namespace jl {
+
+constexpr int kDecTile = 128;    // keys per tile
+constexpr int kDecStages = 3;    // K/V pipeline depth
+constexpr int kDecQRows = 32;    // B operand rows of the score MMA (16 remote + 16 local)
+constexpr int kDecHeads = 16;    // N of the PV MMA (query heads per KV head, padded)
+
+struct DecTcLayout {
+  static constexpr int kTile = kDecTile * 128 * 2;          // 32 KB (K or V tile)
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kDecStages * kTile;
+  static constexpr int kQ = kV + kDecStages * kTile;        // [32][128] bf16 = 8 KB (2 boxes of 4 KB)
+  static constexpr int kP = kQ + kDecQRows * 256;           // 2 x [16][128] bf16 = 2 x 4 KB
+  static constexpr int kRed = kP + 2 * kDecHeads * 256;     // reductions: float [4][16] x 2
+  static constexpr int kBar = kRed + 1024;
+  static constexpr int kBytes = kBar + 512;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 128;  // S^T x2 (64) + O^T (16)
+  static constexpr int kRotWarps = 8;
+  static constexpr int kRotRows = kDecTile / kRotWarps;  // 16 rows per correction warp
+  static constexpr int kThreads = 32 * (6 + kRotWarps);   // 14 warps
+};
+
+struct DecTcBars {
+  uint64_t k_full[kDecStages], k_ready[kDecStages], k_empty[kDecStages];
+  uint64_t v_full[kDecStages], v_empty[kDecStages];
+  uint64_t s_full[2], p_ready[2], pv_done, q_ready, teardown;
+  uint64_t red_full[2], red_end;  // softmax-warp exchanges (bounded, unlike bar.sync)
+  uint32_t tmem_base;
+  int abort;
+};
+
+// warps 2-3 and 8-13 correct keys; 4-7 (one TMEM lane quarter each) run the softmax
+__device__ __forceinline__ int dec_rot_index(int warp) {
+  return warp == 2 ? 0 : warp == 3 ? 1 : (warp >= 8 ? warp - 6 : -1);
+}
+
+// Rotate row r of a swizzled [128][128] bf16 tile in place by R(-n), f = (cos n theta, sin n theta).
+__device__ __forceinline__ void rotate_row_neg(uint8_t* tile, int r, const float (&c)[2], const float (&s)[2],
+                                               int lane) {
+  const int off = r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + ((lane & 3) << 2);
+  __nv_bfloat162* plo = reinterpret_cast<__nv_bfloat162*>(tile + off);
+  __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
+  const float2 a = __bfloat1622float2(*plo);
+  const float2 b = __bfloat1622float2(*phi);
+  float2 ya, yb;
+  ya.x = a.x * c[0] + b.x * s[0];
+  yb.x = b.x * c[0] - a.x * s[0];
+  ya.y = a.y * c[1] + b.y * s[1];
+  yb.y = b.y * c[1] - a.y * s[1];
+  *plo = __float22bfloat162_rn(ya);
+  *phi = __float22bfloat162_rn(yb);
+}
+
+// (c, s) <- (c, s) * e^{i theta} when adv, else unchanged (select, no branch).
+__device__ __forceinline__ void step_factor(float (&c)[2], float (&s)[2], const float (&st_c)[2],
+                                            const float (&st_s)[2], bool adv) {
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float nc = c[e] * st_c[e] - s[e] * st_s[e];
+    const float ns = s[e] * st_c[e] + c[e] * st_s[e];
+    c[e] = adv ? nc : c[e];
+    s[e] = adv ? ns : s[e];
+  }
+}
+
+// Element (row, ch) of a 128-byte-swizzled K-major [rows][128] bf16 operand whose
+// 64-channel boxes are box_bytes apart.
+__device__ __forceinline__ int swz_off(int row, int ch, int box_bytes) {
+  const int cc = ch & 63;
+  return (ch >> 6) * box_bytes + row * 128 + ((((cc * 2) >> 4) ^ (row & 7)) << 4) + ((cc * 2) & 15);
+}
+
+template <int GROUP, bool PLAIN>
+__global__ void __launch_bounds__(DecTcLayout::kThreads, 1)
+    jl_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const DecodeParams p) {
+  using Lay = DecTcLayout;
+  constexpr uint32_t kTileTx = kDecTile * 128 * 2;
+  constexpr uint32_t kIdescS = idesc_bf16_f32(128, kDecQRows, false, false);
+  constexpr uint32_t kIdescO = idesc_bf16_f32(128, kDecHeads, true, false);
+  static_assert(GROUP <= kDecHeads, "up to 16 query heads per KV head");
+
+  const int hk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int L = p.seqlens[b];
+  const int c0 = split * p.chunk;
+  if (c0 >= L) return;
+  if (status_failed()) return;
+  const int c1 = min(c0 + p.chunk, L);
+  const int n_tiles = (c1 - c0 + kDecTile - 1) / kDecTile;
+  const int i = L - 1;
+  int G = 1, jb = -1;  // remote keys are j <= jb
+  if (!PLAIN) {
+    G = max(1, (L + p.w_pre - 1) / p.w_pre);
+    if (G > 1) jb = i - p.w0;
+  }
+  const int64_t row0 = static_cast<int64_t>(b) * p.cache_stride;  // token row of this entry's first key
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sK = smem + Lay::kK;
+  uint8_t* sV = smem + Lay::kV;
+  uint8_t* sQ = smem + Lay::kQ;
+  uint8_t* sP = smem + Lay::kP;
+  float* red = reinterpret_cast<float*>(smem + Lay::kRed);  // [2][4][16]
+  DecTcBars* bars = reinterpret_cast<DecTcBars*>(smem + Lay::kBar);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_ready[s], Lay::kRotWarps);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_ready[t], 128);
+    }
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->q_ready, 128);
+    mbar_init(&bars->teardown, 1);
+    mbar_init(&bars->red_full[0], 128);
+    mbar_init(&bars->red_full[1], 128);
+    mbar_init(&bars->red_end, 128);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int issued[kDecStages] = {0};
+      for (int n = 0; n < n_tiles && !*abort; ++n) {
+        const int s = n % kDecStages;
+        const uint32_t u = n / kDecStages;
+        const int key0 = static_cast<int>(row0) + c0 + n * kDecTile;
+        if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
+        tma_load_3d(sK + s * Lay::kTile, &tm_k, &bars->k_full[s], 0, hk, key0);
+        tma_load_3d(sK + s * Lay::kTile + 16384, &tm_k, &bars->k_full[s], 64, hk, key0);
+        if (u > 0 && !mbar_wait(&bars->v_empty[s], (u - 1) & 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->v_full[s], kTileTx);
+        tma_load_3d(sV + s * Lay::kTile, &tm_v, &bars->v_full[s], 0, hk, key0);
+        tma_load_3d(sV + s * Lay::kTile + 16384, &tm_v, &bars->v_full[s], 64, hk, key0);
+        issued[s] = static_cast<int>(u) + 1;
+      }
+      for (int s = 0; s < kDecStages; ++s)
+        if (issued[s] > 0) {
+          mbar_wait_bounded(&bars->k_full[s], (issued[s] - 1) & 1);
+          mbar_wait_bounded(&bars->v_full[s], (issued[s] - 1) & 1);
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+      auto issue_s = [&](int n) {
+        const uint32_t ka = k_addr + (n % kDecStages) * Lay::kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off_k = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t off_q = (kk >> 2) * (kDecQRows * 128) + (kk & 3) * 32;
+          umma_ss(tmem + (n & 1) * 32, sdesc_kmajor_sw128(ka + off_k), sdesc_kmajor_sw128(q_addr + off_q), kIdescS,
+                  kk > 0);
+        }
+      };
+      auto issue_pv = [&](int n) {
+        const uint32_t va = v_addr + (n % kDecStages) * Lay::kTile;
+        const uint32_t pa = p_addr + (n & 1) * (kDecHeads * 256);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off_p = (kk >> 2) * (kDecHeads * 128) + (kk & 3) * 32;
+          umma_ss(tmem + 64, sdesc_mnmajor_sw128(va + kk * 2048, 16384), sdesc_kmajor_sw128(pa + off_p), kIdescO,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bars->q_ready, 0, abort);
+      if (ok) {
+        tc_fence_after();
+        ok = mbar_wait(&bars->k_ready[0], 0, abort);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        umma_commit(&bars->s_full[0]);
+        umma_commit(&bars->k_empty[0]);
+      }
+      for (int n = 0; n < n_tiles && ok; ++n) {
+        if (n + 1 < n_tiles) {  // scores of the next tile overlap this tile's softmax
+          const int s1 = (n + 1) % kDecStages;
+          if (!(ok = mbar_wait(&bars->k_ready[s1], ((n + 1) / kDecStages) & 1, abort))) break;
+          tc_fence_after();
+          issue_s(n + 1);
+          umma_commit(&bars->s_full[(n + 1) & 1]);
+          umma_commit(&bars->k_empty[s1]);
+        }
+        if (!(ok = mbar_wait(&bars->p_ready[n & 1], (n >> 1) & 1, abort))) break;
+        tc_fence_after();
+        const int s = n % kDecStages;
+        if (!(ok = mbar_wait(&bars->v_full[s], (n / kDecStages) & 1, abort))) break;
+        issue_pv(n);
+        umma_commit(&bars->pv_done);
+        umma_commit(&bars->v_empty[s]);
+      }
+      umma_commit(&bars->teardown);
+      mbar_wait_bounded(&bars->teardown, 0);
+    }
+  } else if (dec_rot_index(warp) >= 0) {
+    // ---------------------------------------------------- correction warps
+    const int rw = dec_rot_index(warp);
+    float st_c[2], st_s[2];  // e^{i theta_c}
+    {
+      const float2 cc = __ldg(reinterpret_cast<const float2*>(p.cos_tab + 64 + 2 * lane));
+      const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + 64 + 2 * lane));
+      st_c[0] = cc.x; st_c[1] = cc.y; st_s[0] = ss.x; st_s[1] = ss.y;
+    }
+    auto anchor = [&](int n, float (&c)[2], float (&s)[2]) {
+      const int j = c0 + n * kDecTile + Lay::kRotRows * rw;
+      int64_t row = j - j / G;  // correction index n_j = j - f(j)
+      row = row > p.n_tab_rows - 1 ? p.n_tab_rows - 1 : row;
+      const float2 cc = __ldg(reinterpret_cast<const float2*>(p.cos_tab + row * 64 + 2 * lane));
+      const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + row * 64 + 2 * lane));
+      c[0] = cc.x; c[1] = cc.y; s[0] = ss.x; s[1] = ss.y;
+    };
+    float nc[2], ns[2];
+    anchor(0, nc, ns);
+    for (int n = 0; n < n_tiles; ++n) {
+      float fc[2] = {nc[0], nc[1]}, fs[2] = {ns[0], ns[1]};
+      if (n + 1 < n_tiles) anchor(n + 1, nc, ns);
+      const int s = n % kDecStages;
+      if (!mbar_wait(&bars->k_full[s], (n / kDecStages) & 1, abort)) break;
+      const int j0 = c0 + n * kDecTile + Lay::kRotRows * rw;  // key of this warp's first row
+      const int last_remote = min(jb, c1 - 1) - j0;             // rows r <= last_remote are remote
+      if (last_remote >= 0) {
+        uint8_t* slice = sK + s * Lay::kTile + Lay::kRotRows * rw * 128;
+        int cnt = j0 % G;
+        // Straight-line rows: the factor steps by e^{i theta} except where f steps
+        // up (then n_j stays), chosen with selects, not branches.
+        if (last_remote >= Lay::kRotRows - 1) {
+#pragma unroll
+          for (int r = 0; r < Lay::kRotRows; ++r) {
+            rotate_row_neg(slice, r, fc, fs, lane);
+            cnt = (cnt + 1 == G) ? 0 : cnt + 1;
+            step_factor(fc, fs, st_c, st_s, cnt != 0);
+          }
+        } else {  // the slice straddles the window edge: rows past last_remote stay as cached
+#pragma unroll
+          for (int r = 0; r < Lay::kRotRows; ++r) {
+            if (r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
+            cnt = (cnt + 1 == G) ? 0 : cnt + 1;
+            step_factor(fc, fs, st_c, st_s, cnt != 0);
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->k_ready[s]);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int wq = warp - 4;  // 0..3: TMEM lane quarter
+    const int tid = threadIdx.x - 128;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
+    // Query operand: rows 0..15 remote-corrected R(f(i) - i) q~, rows 16..31 q~; zero padding.
+    {
+      const int nq = i - i / G;
+      for (int e = tid; e < kDecQRows * 64; e += 128) {
+        const int row = e >> 6, c = e & 63;
+        const int g = row & 15;
+        float lo = 0.f, hi = 0.f;
+        if (g < GROUP) {
+          const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * GROUP + g) * 128;
+          lo = __bfloat162float(qp[c]);
+          hi = __bfloat162float(qp[c + 64]);
+          if (row < 16 && G > 1 && !PLAIN) {
+            const float cs = p.cos_tab[static_cast<int64_t>(nq) * 64 + c];
+            const float sn = p.sin_tab[static_cast<int64_t>(nq) * 64 + c];
+            const float a = lo, bb = hi;
+            lo = a * cs + bb * sn;
+            hi = bb * cs - a * sn;
+          }
+        }
+        *reinterpret_cast<__nv_bfloat16*>(sQ + swz_off(row, c, kDecQRows * 128)) = __float2bfloat16_rn(lo);
+        *reinterpret_cast<__nv_bfloat16*>(sQ + swz_off(row, c + 64, kDecQRows * 128)) = __float2bfloat16_rn(hi);
+      }
+      // both P buffers start at zero (rows >= GROUP are never written)
+      for (int e = tid; e < 2 * kDecHeads * 256 / 16; e += 128)
+        reinterpret_cast<uint4*>(sP)[e] = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->q_ready);
+    }
+    float m_run[GROUP], l_part[GROUP];
+#pragma unroll
+    for (int g = 0; g < GROUP; ++g) {
+      m_run[g] = -INFINITY;
+      l_part[g] = 0.f;
+    }
+    bool ok = true;
+    for (int n = 0; n < n_tiles && ok; ++n) {
+      if (!(ok = mbar_wait(&bars->s_full[n & 1], (n >> 1) & 1, abort))) break;
+      tc_fence_after();
+      uint32_t sr[32];
+      tmem_ld32(t_lane + (n & 1) * 32, sr);
+      const int j = c0 + n * kDecTile + tid;  // this thread's key
+      const bool valid = j < c1;
+      const bool rem = j <= jb;
+      float sv[GROUP];
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g)
+        sv[g] = valid ? __uint_as_float(sr[rem ? g : 16 + g]) : -INFINITY;
+      // per-head tile maximum over the 128 keys
+      float* rb = red + (n & 1) * 64;
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        float x = sv[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+        if (lane == 0) rb[wq * 16 + g] = x;
+      }
+      mbar_arrive(&bars->red_full[n & 1]);
+      if (!(ok = mbar_wait(&bars->red_full[n & 1], (n >> 1) & 1, abort))) break;
+      float alpha[GROUP];
+      bool any_resc = false;
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        const float mt = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g])) * sl2;
+        const float m_new = fmaxf(m_run[g], mt);
+        const bool resc = (m_run[g] != -INFINITY) && (m_new > m_run[g] + 8.f);
+        alpha[g] = resc ? ex2_approx(m_run[g] - m_new) : 1.f;
+        any_resc |= resc;
+        if (resc || m_run[g] == -INFINITY) m_run[g] = m_new;
+      }
+      // PV(n-1) must be complete before P buffer (n & 1) is rewritten and before O is rescaled
+      if (n > 0 && !(ok = mbar_wait(&bars->pv_done, (n - 1) & 1, abort))) break;
+      tc_fence_after();
+      uint8_t* pb = sP + (n & 1) * (kDecHeads * 256);
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        const float m_use = (m_run[g] == -INFINITY) ? 0.f : m_run[g];
+        const float pr = valid ? ex2_approx(fmaf(sv[g], sl2, -m_use)) : 0.f;
+        l_part[g] = l_part[g] * alpha[g] + pr;
+        *reinterpret_cast<__nv_bfloat16*>(pb + swz_off(g, tid, kDecHeads * 128)) = __float2bfloat16_rn(pr);
+      }
+      if (any_resc && n > 0) {  // uniform: every thread computed the same alphas
+        uint32_t o[32];
+        tmem_ld32(t_lane + 64, o);  // columns 64..95; the first 16 are O^T
+#pragma unroll
+        for (int g = 0; g < GROUP; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+        tmem_st32(t_lane + 64, o);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready[n & 1]);
+    }
+    // epilogue: row sums across the 128 threads, then the partial per query head
+    if (ok && mbar_wait(&bars->pv_done, (n_tiles - 1) & 1, abort)) {
+      tc_fence_after();
+      float* rl = red + 128;  // [4][16]
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        float x = l_part[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (lane == 0) rl[wq * 16 + g] = x;
+      }
+      mbar_arrive(&bars->red_end);
+      if (mbar_wait(&bars->red_end, 0, abort)) {
+      uint32_t o[32];
+      tmem_ld32(t_lane + 64, o);  // thread = channel tid
+      float* ws = p.ws + ((static_cast<int64_t>(b) * p.n_split + split) * p.Hq + hk * GROUP) * (128 + 2);
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        float* dst = ws + static_cast<int64_t>(g) * (128 + 2);
+        dst[2 + tid] = __uint_as_float(o[g]);
+        if (tid == 0) {
+          dst[0] = m_run[g];
+          dst[1] = rl[g] + rl[16 + g] + rl[32 + g] + rl[48 + g];
+        }
+      }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+}  // namespace jl

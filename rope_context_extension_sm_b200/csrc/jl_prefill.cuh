@@ -205,12 +205,18 @@ __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, in
                                              const RotFactor<D>& st, int lane) {
   int cnt = (base + 32 * rw) % g;
   uint8_t* slice = tile + 32 * rw * 128;  // 32 rows x 128 B; row & 7 == r & 7
-#pragma unroll 4
+#pragma unroll 8
   for (int r = 0; r < 32; ++r) {
     rotate_row<D>(slice, r, f, lane);
-    if (++cnt == g) {
-      cnt = 0;
-      advance<D>(f, st);
+    // the position (base) or remote position (f(pos)) steps up every g rows;
+    // select, not branch, so the rows stay one straight-line block
+    cnt = (cnt + 1 == g) ? 0 : cnt + 1;
+    RotFactor<D> nf = f;
+    advance<D>(nf, st);
+#pragma unroll
+    for (int e = 0; e < RotFactor<D>::NF; ++e) {
+      f.c[e] = cnt == 0 ? nf.c[e] : f.c[e];
+      f.s[e] = cnt == 0 ? nf.s[e] : f.s[e];
     }
   }
 }
