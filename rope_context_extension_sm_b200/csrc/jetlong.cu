@@ -155,9 +155,11 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
 bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) { return head_dim == 128 && Hq / Hkv <= 16; }
 
 // Keys per split.  CUDA-core kernel: a power of two in [64, 512].  Tensor-core
-// kernel: whole 128-key tiles, sized so that 8 KV heads x B entries give about
-// four waves of CTAs (the split count depends only on B and max_seqlen, never on
-// the head counts, so the workspace-size query below can bound it).
+// kernel: whole 128-key tiles, sized so that 8 KV heads x B entries fill the 148
+// SMs of a B200 in one wave (one CTA per SM; a single wave keeps each CTA's
+// K/V pipeline full instead of paying a cold start per short chunk).  The split
+// count depends only on B and max_seqlen, never on the head counts, so the
+// workspace-size query below can bound it.
 int chunk_cuda_core(int32_t max_seqlen) {
   int c = 64;
   while (c < 512 && static_cast<int64_t>(c) * 256 < max_seqlen) c *= 2;
@@ -166,7 +168,7 @@ int chunk_cuda_core(int32_t max_seqlen) {
 
 int chunk_tc(int32_t B, int32_t max_seqlen) {
   const int64_t tiles = (static_cast<int64_t>(max_seqlen) + jl::kDecTile - 1) / jl::kDecTile;
-  const int64_t want_ctas = 148 * 4;
+  const int64_t want_ctas = 148;
   int64_t per = (tiles * 8 * B + want_ctas - 1) / want_ctas;
   per = per < 1 ? 1 : per;
   return static_cast<int>(per * jl::kDecTile);
@@ -174,7 +176,7 @@ int chunk_tc(int32_t B, int32_t max_seqlen) {
 
 template <int GROUP, bool PLAIN>
 jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) {
-  using Lay = jl::DecTcLayout;
+  using Lay = jl::DecTcLayout<GROUP>;
   CUtensorMap tk, tv;
   jl_status s;
   const int64_t rows = static_cast<int64_t>(B) * prm.cache_stride;

@@ -10,8 +10,9 @@
 // CTA = (KV head, chunk of keys, batch entry).  Per 128-key tile:
 //   warp 0      TMA producer: raw K and V tiles (3 stages)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-3,  correction warps: rotate the remote rows of the K tile in place
-//   8-13        by R(-(j - f(j))) (cos/sin stepped along the rows by complex
+//   warps 2-3,  correction warps (16, or 8 for 16 heads per KV head): rotate
+//   8..         the remote rows of the K tile in place by R(-(j - f(j)))
+//               (cos/sin stepped along the rows by complex
 //               multiplication, anchored on a table row prefetched a tile ahead)
 //   warps 4-7   softmax, thread = key row of S^T and channel row of O^T
 // MMAs:  S^T[128 keys x 32] = K_tile . [R(f(i)-i) q~ (16 rows) | q~ (16 rows)]^T
@@ -33,6 +34,7 @@ constexpr int kDecStages = 3;    // K/V pipeline depth
 constexpr int kDecQRows = 32;    // B operand rows of the score MMA (16 remote + 16 local)
 constexpr int kDecHeads = 16;    // N of the PV MMA (query heads per KV head, padded)
 
+template <int GROUP>
 struct DecTcLayout {
   static constexpr int kTile = kDecTile * 128 * 2;          // 32 KB (K or V tile)
   static constexpr int kK = 0;
@@ -44,9 +46,11 @@ struct DecTcLayout {
   static constexpr int kBytes = kBar + 512;
   static constexpr int kAlloc = kBytes + 1024;
   static constexpr uint32_t kTmemCols = 128;  // S^T x2 (64) + O^T (16)
-  static constexpr int kRotWarps = 8;
-  static constexpr int kRotRows = kDecTile / kRotWarps;  // 16 rows per correction warp
-  static constexpr int kThreads = 32 * (6 + kRotWarps);   // 14 warps
+  // correction warps: 16 (8 rows each) unless 16 query heads per KV head make the
+  // softmax warps register-heavy, then 8 (16 rows each)
+  static constexpr int kRotWarps = GROUP <= 8 ? 16 : 8;
+  static constexpr int kRotRows = kDecTile / kRotWarps;
+  static constexpr int kThreads = 32 * (6 + kRotWarps);
 };
 
 struct DecTcBars {
@@ -58,7 +62,7 @@ struct DecTcBars {
   int abort;
 };
 
-// warps 2-3 and 8-13 correct keys; 4-7 (one TMEM lane quarter each) run the softmax
+// warps 2-3 and 8.. correct keys; 4-7 (one TMEM lane quarter each) run the softmax
 __device__ __forceinline__ int dec_rot_index(int warp) {
   return warp == 2 ? 0 : warp == 3 ? 1 : (warp >= 8 ? warp - 6 : -1);
 }
@@ -100,10 +104,10 @@ __device__ __forceinline__ int swz_off(int row, int ch, int box_bytes) {
 }
 
 template <int GROUP, bool PLAIN>
-__global__ void __launch_bounds__(DecTcLayout::kThreads, 1)
+__global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     jl_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p) {
-  using Lay = DecTcLayout;
+  using Lay = DecTcLayout<GROUP>;
   constexpr uint32_t kTileTx = kDecTile * 128 * 2;
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, kDecQRows, false, false);
   constexpr uint32_t kIdescO = idesc_bf16_f32(128, kDecHeads, true, false);
