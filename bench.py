@@ -171,12 +171,18 @@ def _barrier(world):
     torch.cuda.synchronize()
 
 
-def _max_over_ranks(x, world):
+def _max_over_ranks(x, world, device="cuda"):
+    """Max of a per-rank device time over all ranks (the slowest rank sets the step time)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(world, units_per_rank, steps, max_total_ms):
+    """Whole-job throughput of N independent replicas: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank * steps / (max_total_ms * 1e-3)
 
 
 # --------------------------------------------------------------- our arm ----
@@ -253,7 +259,7 @@ def run_ours(args, world, rank, local):
     dec_avg = _max_over_ranks(sum(dec_ms) / K, world)
 
     flops = PREFILL.useful_flops()
-    value = world * flops * K / (total_ms * 1e-3) / 1e12  # whole job, prefill flops over the step time
+    value = replica_throughput(world, flops, K, total_ms) / 1e12  # whole job, prefill flops over the step time
     prefill_tflops = flops / (pre_avg * 1e-3) / 1e12
     burst, sustained, hbm, peak_kind = _peaks()
     kv_bytes = 2 * DECODE_L * DECODE.n_kv_heads * DECODE.head_dim * 2

@@ -63,6 +63,18 @@ int64_t jl_group_size(int64_t L, int64_t w_pretrained);
 jl_status jl_sync_status(jl_stream_t stream);
 
 /*
+ * Failure-detection self-test (no counterpart in the paper; it exercises this
+ * library's bounded waits).  Launches one thread that waits on a shared-memory
+ * barrier that nothing ever completes, giving up after limit_cycles SM clock
+ * cycles: the kernel records JL_ERR_TIMEOUT in the device status word and
+ * returns normally, so no GPU fault or hang is involved.  A following
+ * jl_sync_status() reports JL_ERR_TIMEOUT and clears the word; until then,
+ * later launches of the attention kernels see the word and skip their work.
+ * limit_cycles must be in [1000, 2000000000].
+ */
+jl_status jl_selftest_wait_timeout(int64_t limit_cycles, jl_stream_t stream);
+
+/*
  * RoPE cos/sin tables.  Fills cos_out[p][c] = cos(p * theta_c) and
  * sin_out[p][c] = sin(p * theta_c) for p in [0, n_pos), c in [0, head_dim/2),
  * row-major fp32 [n_pos][head_dim/2].  Angles and cos/sin are computed in fp64

@@ -333,6 +333,15 @@ jl_status jl_sync_status(jl_stream_t stream) {
   return ok();
 }
 
+jl_status jl_selftest_wait_timeout(int64_t limit_cycles, jl_stream_t stream) {
+  if (limit_cycles < 1000 || limit_cycles > 2000000000LL)
+    return fail(JL_ERR_INVALID, "limit_cycles must be in [1000, 2e9] (got %lld)", (long long)limit_cycles);
+  jl::jl_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ok();
+}
+
 jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
                          jl_stream_t stream) {
   if (!cos_out || !sin_out) return fail(JL_ERR_INVALID, "null table pointer");

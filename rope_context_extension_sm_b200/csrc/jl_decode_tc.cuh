@@ -96,6 +96,39 @@ __device__ __forceinline__ void step_factor(float (&c)[2], float (&s)[2], const 
   }
 }
 
+// Correct the remote rows (r <= last_remote) of an ROWS-row slice of keys j0 ..:
+// R(-n_j), n_j = j - floor(j / G).  n steps by one per row except where f steps up
+// (row r with (j0 + r + 1) % G == 0).  GS = G in {2, 4, 8} with j0 % G == 0 makes
+// those rows compile-time; GS = 0 keeps a counter and selects.
+template <int ROWS, int GS>
+__device__ __forceinline__ void correct_slice(uint8_t* slice, int j0, int G, int last_remote, bool full,
+                                              float (&fc)[2], float (&fs)[2], const float (&st_c)[2],
+                                              const float (&st_s)[2], int lane) {
+  if constexpr (GS > 0) {
+    if (full) {
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        rotate_row_neg(slice, r, fc, fs, lane);
+        if ((r + 1) % GS != 0) step_factor(fc, fs, st_c, st_s, true);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        if (r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
+        if ((r + 1) % GS != 0) step_factor(fc, fs, st_c, st_s, true);
+      }
+    }
+  } else {
+    int cnt = j0 % G;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      if (full || r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
+      cnt = (cnt + 1 == G) ? 0 : cnt + 1;
+      step_factor(fc, fs, st_c, st_s, cnt != 0);
+    }
+  }
+}
+
 // Element (row, ch) of a 128-byte-swizzled K-major [rows][128] bf16 operand whose
 // 64-channel boxes are box_bytes apart.
 __device__ __forceinline__ int swz_off(int row, int ch, int box_bytes) {
@@ -278,23 +311,12 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       const int last_remote = min(jb, c1 - 1) - j0;             // rows r <= last_remote are remote
       if (last_remote >= 0) {
         uint8_t* slice = sK + s * Lay::kTile + Lay::kRotRows * rw * 128;
-        int cnt = j0 % G;
-        // Straight-line rows: the factor steps by e^{i theta} except where f steps
-        // up (then n_j stays), chosen with selects, not branches.
-        if (last_remote >= Lay::kRotRows - 1) {
-#pragma unroll
-          for (int r = 0; r < Lay::kRotRows; ++r) {
-            rotate_row_neg(slice, r, fc, fs, lane);
-            cnt = (cnt + 1 == G) ? 0 : cnt + 1;
-            step_factor(fc, fs, st_c, st_s, cnt != 0);
-          }
-        } else {  // the slice straddles the window edge: rows past last_remote stay as cached
-#pragma unroll
-          for (int r = 0; r < Lay::kRotRows; ++r) {
-            if (r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
-            cnt = (cnt + 1 == G) ? 0 : cnt + 1;
-            step_factor(fc, fs, st_c, st_s, cnt != 0);
-          }
+        const bool full = last_remote >= Lay::kRotRows - 1;  // else the slice straddles the window edge
+        switch (G) {  // slices start at multiples of 8 keys: for G | 8 the step rows are fixed
+          case 2: correct_slice<Lay::kRotRows, 2>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
+          case 4: correct_slice<Lay::kRotRows, 4>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
+          case 8: correct_slice<Lay::kRotRows, 8>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
+          default: correct_slice<Lay::kRotRows, 0>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
         }
         fence_proxy_async_smem();
       }

@@ -200,24 +200,47 @@ __device__ __forceinline__ int64_t slice_anchor_row(int base, int rw, int g) {
 // Rotate rows [32 rw, 32 rw + 32) of a tile whose row r sits at position base + r:
 // by R(pos) when g == 1, by R(floor(pos / g)) otherwise.  f is the factor of the
 // slice's first row; the remote position advances by one every g rows.
-template <int D>
+// Rotate rows [32 rw, 32 rw + 32) of a tile whose row r sits at position base + r:
+// by R(pos) when g == 1, by R(floor(pos / g)) otherwise.  f is the factor of the
+// slice's first row; the (remote) position steps up every g rows.  Tile bases are
+// multiples of 128 and slices start at multiples of 32, so for GS = g in {1, 2, 4}
+// the slice starts on a group boundary and the step rows are known at compile
+// time; GS = 0 handles any g with a running counter and selects.
+template <int D, int GS>
 __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, int g, RotFactor<D> f,
                                              const RotFactor<D>& st, int lane) {
-  int cnt = (base + 32 * rw) % g;
   uint8_t* slice = tile + 32 * rw * 128;  // 32 rows x 128 B; row & 7 == r & 7
+  if constexpr (GS > 0) {
 #pragma unroll 8
-  for (int r = 0; r < 32; ++r) {
-    rotate_row<D>(slice, r, f, lane);
-    // the position (base) or remote position (f(pos)) steps up every g rows;
-    // select, not branch, so the rows stay one straight-line block
-    cnt = (cnt + 1 == g) ? 0 : cnt + 1;
-    RotFactor<D> nf = f;
-    advance<D>(nf, st);
-#pragma unroll
-    for (int e = 0; e < RotFactor<D>::NF; ++e) {
-      f.c[e] = cnt == 0 ? nf.c[e] : f.c[e];
-      f.s[e] = cnt == 0 ? nf.s[e] : f.s[e];
+    for (int r = 0; r < 32; ++r) {
+      rotate_row<D>(slice, r, f, lane);
+      if ((r + 1) % GS == 0) advance<D>(f, st);
     }
+  } else {
+    int cnt = (base + 32 * rw) % g;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      rotate_row<D>(slice, r, f, lane);
+      cnt = (cnt + 1 == g) ? 0 : cnt + 1;
+      RotFactor<D> nf = f;
+      advance<D>(nf, st);
+#pragma unroll
+      for (int e = 0; e < RotFactor<D>::NF; ++e) {
+        f.c[e] = cnt == 0 ? nf.c[e] : f.c[e];
+        f.s[e] = cnt == 0 ? nf.s[e] : f.s[e];
+      }
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void rotate_slice_any(uint8_t* tile, int rw, int base, int g, const RotFactor<D>& f,
+                                                 const RotFactor<D>& st, int lane) {
+  switch (g) {
+    case 1: rotate_slice<D, 1>(tile, rw, base, g, f, st, lane); break;
+    case 2: rotate_slice<D, 2>(tile, rw, base, g, f, st, lane); break;
+    case 4: rotate_slice<D, 4>(tile, rw, base, g, f, st, lane); break;
+    default: rotate_slice<D, 0>(tile, rw, base, g, f, st, lane); break;
   }
 }
 
@@ -444,7 +467,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         RotFactor<D> fq;
         load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane);
         if (!mbar_wait(&bars->q_full, n == 0 ? 0 : 1, abort)) break;
-        for (int t = 0; t < NQT; ++t) rotate_slice<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, step, lane);
+        for (int t = 0; t < NQT; ++t) rotate_slice_any<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, step, lane);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_ready);
@@ -453,7 +476,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (n + 1 < sc.n_virt) load_factor<D>(fk_next, p, key_anchor(n + 1), lane);  // prefetch a tile ahead
       const int s = n % kStages;
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
-      rotate_slice<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
+      rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);

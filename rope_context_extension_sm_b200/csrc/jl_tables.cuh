@@ -23,4 +23,24 @@ __global__ void __launch_bounds__(256) jl_rope_table_kernel(float* __restrict__ 
   }
 }
 
+// Waits on a barrier nobody arrives at, for at most `limit` cycles, then records
+// a timeout exactly as the attention kernels' bounded waits do.
+__global__ void jl_selftest_wait_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (clock64() - t0 > limit) {
+        atomicOr(&g_status, kDevErrTimeout);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace jl

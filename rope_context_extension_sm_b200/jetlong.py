@@ -48,6 +48,7 @@ SIGNATURES = {
     "jl_bifocal_decode_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
                                                  _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
+    "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -100,6 +101,11 @@ def jl_group_size(L: int, w_pretrained: int) -> int:
 def jl_sync_status(stream=None) -> None:
     """Synchronise the stream and raise JetLongError if a kernel's bounded wait ran out."""
     _check(_lib.jl_sync_status(_stream(stream)), "jl_sync_status")
+
+
+def jl_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Launch the bounded-wait self-test; jl_sync_status() then raises JL_ERR_TIMEOUT."""
+    _check(_lib.jl_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "jl_selftest_wait_timeout")
 
 
 def jl_rope_tables(n_pos: int, head_dim: int, rope_base: float, *, device="cuda", cos=None, sin=None, stream=None):

@@ -102,3 +102,8 @@ def test_rope_tables_rejects_bad_arguments(jlmod):
     assert jlmod._lib.jl_rope_tables(16, 16, 10, 100, 1e4, None) == 2
     assert jlmod._lib.jl_rope_tables(None, 16, 10, 128, 1e4, None) == 1
     assert jlmod._lib.jl_rope_tables(16, 16, 10, 128, 0.5, None) == 1
+
+
+def test_selftest_rejects_bad_limits(jlmod):
+    assert jlmod._lib.jl_selftest_wait_timeout(10, None) == 1
+    assert jlmod._lib.jl_selftest_wait_timeout(3_000_000_000, None) == 1

@@ -91,6 +91,19 @@ def test_rope_tables_match_fp64_rounded_once(jl, n, d, base):
         assert (g != ref.astype(np.float32)).mean() < 1e-3
 
 
+# --------------------------------------------------------- failure detection ----
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable(jl):
+    """A wait that nothing completes ends after its limit with JL_ERR_TIMEOUT (no trap,
+    no hang); jl_sync_status reports and clears it; the context keeps working."""
+    jl.jl_selftest_wait_timeout(2_000_000)
+    with pytest.raises(jl.JetLongError) as err:
+        jl.jl_sync_status()
+    assert err.value.status == jl.JL_ERR_TIMEOUT
+    jl.jl_sync_status()  # cleared
+    _compare_all_rows(jl, I.TINY)
+
+
 # ----------------------------------------------------------------- prefill ----
 
 def test_tiny_prefill_all_rows(jl):
