@@ -59,7 +59,9 @@ const char* jl_last_error(void);
 int64_t jl_group_size(int64_t L, int64_t w_pretrained);
 
 /* Synchronises `stream`, then returns and clears the device status word:
- * JL_OK, JL_ERR_TIMEOUT, or JL_ERR_CUDA if the synchronisation itself failed. */
+ * JL_OK; JL_ERR_TIMEOUT if a bounded wait ran out; JL_ERR_INVALID if a cache
+ * writer met a position outside the cache or the tables; JL_ERR_CUDA if the
+ * synchronisation itself failed. */
 jl_status jl_sync_status(jl_stream_t stream);
 
 /*
@@ -162,6 +164,39 @@ jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cach
                           int32_t head_dim, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
                           float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                           jl_stream_t stream);
+
+/*
+ * Base-RoPE KV cache writers (Methodology section 2: the cache holds the
+ * un-compressed base keys R(j) k_j at their absolute positions and is written
+ * once per token; the bifocal decode only reads it).
+ *
+ * jl_kv_cache_fill: for every prompt token t of packed sequence b (position
+ * p = t - cu_seqlens[b]), k_cache[b][p] = R(p) k[t] (fp32 math, rounded to
+ * bf16) and v_cache[b][p] = v[t], for every KV head.
+ *   k, v        bf16 [total_tokens][Hkv][head_dim], k RAW
+ *   cu_seqlens  device int32 [batch + 1] as for jl_bifocal_prefill
+ *   k_cache, v_cache  bf16 [batch][cache_stride][Hkv][head_dim]
+ * A position >= cache_stride or >= n_tab_rows is skipped and reported by
+ * jl_sync_status() as JL_ERR_INVALID (the lengths live on the device).
+ */
+jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                           int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+                           const float* sin_tab, int64_t n_tab_rows, void* k_cache, void* v_cache,
+                           int64_t cache_stride, jl_stream_t stream);
+
+/*
+ * One decode step's inputs: entry b's new token sits at i = seqlens[b] - 1
+ * (seqlens already counts it).  q_out[b] = R(i) q[b] (the base-rotated query
+ * jl_bifocal_decode takes), k_cache[b][i] = R(i) k[b], v_cache[b][i] = v[b].
+ *   q      bf16 [B][Hq][head_dim] raw;  k, v  bf16 [B][Hkv][head_dim], k raw
+ *   q_out  bf16 [B][Hq][head_dim];  caches as for jl_bifocal_decode (written
+ *          only at position i)
+ * Out-of-range positions are skipped and reported like jl_kv_cache_fill.
+ */
+jl_status jl_decode_append(const void* q, const void* k, const void* v, const int32_t* seqlens, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t head_dim, const float* cos_tab, const float* sin_tab,
+                           int64_t n_tab_rows, void* q_out, void* k_cache, void* v_cache, int64_t cache_stride,
+                           jl_stream_t stream);
 
 /*
  * jl_bifocal_decode without a caller workspace.  The paper has no counterpart:

@@ -13,6 +13,7 @@
 #include <string>
 
 #include "jetlong.h"
+#include "jl_append.cuh"
 #include "jl_decode.cuh"
 #include "jl_decode_tc.cuh"
 #include "jl_prefill.cuh"
@@ -329,6 +330,8 @@ jl_status jl_sync_status(jl_stream_t stream) {
     e = cudaMemcpyToSymbol(jl::g_status, &zero, sizeof zero);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
     if (word & jl::kDevErrTimeout) return fail(JL_ERR_TIMEOUT, "a bounded in-kernel wait ran out");
+    if (word & jl::kDevErrBounds)
+      return fail(JL_ERR_INVALID, "a cache writer met a position outside the cache or the RoPE tables");
   }
   return ok();
 }
@@ -376,6 +379,76 @@ jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const in
                            void* out, float* lse, jl_stream_t stream) {
   return prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, 0, 1, 1, cos_tab,
                         sin_tab, n_tab_rows, softmax_scale, out, lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                           int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+                           const float* sin_tab, int64_t n_tab_rows, void* k_cache, void* v_cache,
+                           int64_t cache_stride, jl_stream_t stream) {
+  if (batch < 0 || total_tokens < 0 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1)
+    return fail(JL_ERR_INVALID, "need batch >= 0, total_tokens >= 0, Hkv >= 1, cache_stride >= 1, n_tab_rows >= 1");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (batch == 0 || total_tokens == 0) return ok();
+  if (!k || !v || !cu_seqlens || !cos_tab || !sin_tab || !k_cache || !v_cache)
+    return fail(JL_ERR_INVALID, "null pointer argument");
+  jl::AppendParams prm{};
+  prm.k = static_cast<const __nv_bfloat16*>(k);
+  prm.v = static_cast<const __nv_bfloat16*>(v);
+  prm.lens = cu_seqlens;
+  prm.cos_tab = cos_tab;
+  prm.sin_tab = sin_tab;
+  prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  prm.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  prm.total_tokens = total_tokens;
+  prm.cache_stride = cache_stride;
+  prm.n_tab_rows = n_tab_rows;
+  prm.batch = batch;
+  prm.Hkv = Hkv;
+  const int64_t rows = total_tokens * Hkv;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (head_dim == 128) jl::jl_kv_fill_kernel<128><<<blocks, 256, 0, st>>>(prm);
+  else jl::jl_kv_fill_kernel<64><<<blocks, 256, 0, st>>>(prm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kv fill launch");
+  return ok();
+}
+
+jl_status jl_decode_append(const void* q, const void* k, const void* v, const int32_t* seqlens, int32_t B,
+                           int32_t Hq, int32_t Hkv, int32_t head_dim, const float* cos_tab, const float* sin_tab,
+                           int64_t n_tab_rows, void* q_out, void* k_cache, void* v_cache, int64_t cache_stride,
+                           jl_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1)
+    return fail(JL_ERR_INVALID, "need B >= 0, Hq >= 1, Hkv >= 1, cache_stride >= 1, n_tab_rows >= 1");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (B == 0) return ok();
+  if (!q || !k || !v || !seqlens || !cos_tab || !sin_tab || !q_out || !k_cache || !v_cache)
+    return fail(JL_ERR_INVALID, "null pointer argument");
+  jl::AppendParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k);
+  prm.v = static_cast<const __nv_bfloat16*>(v);
+  prm.lens = seqlens;
+  prm.cos_tab = cos_tab;
+  prm.sin_tab = sin_tab;
+  prm.q_out = static_cast<__nv_bfloat16*>(q_out);
+  prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  prm.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  prm.cache_stride = cache_stride;
+  prm.n_tab_rows = n_tab_rows;
+  prm.batch = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  const int64_t rows = static_cast<int64_t>(B) * (Hq + Hkv);
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (head_dim == 128) jl::jl_decode_append_kernel<128><<<blocks, 256, 0, st>>>(prm);
+  else jl::jl_decode_append_kernel<64><<<blocks, 256, 0, st>>>(prm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
+  return ok();
 }
 
 size_t jl_bifocal_decode_workspace_size(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {

@@ -49,6 +49,10 @@ SIGNATURES = {
                                                  _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
     "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
+    "jl_kv_cache_fill": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _i64,
+                                        _vp]),
+    "jl_decode_append": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
+                                        _i64, _vp]),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -163,6 +167,35 @@ def jl_plain_prefill(q, k, v, cu_seqlens, max_seqlen: int, cos, sin, *, softmax_
                                  _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out), _ptr(lse),
                                  _stream(stream)), "jl_plain_prefill")
     return out, lse
+
+
+def jl_kv_cache_fill(k, v, cu_seqlens, cos, sin, k_cache, v_cache, *, stream=None):
+    """Write R(p) k and v of every prompt token into base-RoPE caches [B][stride][Hkv][d]."""
+    _need(k, torch.bfloat16, "k", 3)
+    _need(v, torch.bfloat16, "v", 3)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    T, hkv, d = k.shape
+    _check(_lib.jl_kv_cache_fill(_ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.shape[0] - 1, T, hkv, d, _ptr(cos),
+                                 _ptr(sin), cos.shape[0], _ptr(k_cache), _ptr(v_cache), k_cache.shape[1],
+                                 _stream(stream)), "jl_kv_cache_fill")
+    return k_cache, v_cache
+
+
+def jl_decode_append(q, k, v, seqlens, cos, sin, k_cache, v_cache, *, q_out=None, stream=None):
+    """Rotate one new raw token per entry by R(seqlens-1): returns q~ and appends k~, v to the caches."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k, torch.bfloat16, "k", 3)
+    _need(v, torch.bfloat16, "v", 3)
+    _need(seqlens, torch.int32, "seqlens", 1)
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    B, hq, d = q.shape
+    _check(_lib.jl_decode_append(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, hq, k.shape[1], d, _ptr(cos),
+                                 _ptr(sin), cos.shape[0], _ptr(q_out), _ptr(k_cache), _ptr(v_cache),
+                                 k_cache.shape[1], _stream(stream)), "jl_decode_append")
+    return q_out
 
 
 def jl_bifocal_decode_workspace_size(B: int, Hq: int, head_dim: int, max_seqlen: int) -> int:

@@ -304,3 +304,67 @@ def test_decode_walk_across_G_boundary(jl):
         out, lse = _run_decode(jl, cfg, q_t[None], kd, vd, [L], max_len, cos, sin)
         ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
         _check(out[0], lse[0], ro, rl, f"walk step {t} (L={L}, G={O.group_size(L, cfg.w_pretrained)})")
+
+
+# ------------------------------------------------- KV cache writers (append) ----
+
+def test_kv_cache_fill_writes_base_rope_keys(jl):
+    """cache[b][p] = R(p) k (fp32 math, one bf16 rounding) and v copied, for packed varlen prompts."""
+    cfg = I.PrefillConfig("fill", (300, 1, 129, 0, 64), 4, 2, 128, 32, 64, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    stride = 320
+    kc = torch.zeros((len(cfg.seqlens), stride, 2, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    cos, sin = _tables(jl, stride, 128, cfg.rope_base)
+    jl.jl_kv_cache_fill(k.cuda(), v.cuda(), cu.cuda(), cos, sin, kc, vc)
+    jl.jl_sync_status()
+    kc, vc = kc.cpu(), vc.cpu()
+    for b, L in enumerate(cfg.seqlens):
+        s0 = int(cu[b])
+        if L == 0:
+            continue
+        pos = np.repeat(np.arange(L), 2)
+        ref = O.rotate_rows(k[s0:s0 + L].float().numpy().reshape(-1, 128), pos, cfg.rope_base).reshape(L, 2, 128)
+        got = kc[b, :L].float().numpy()
+        np.testing.assert_allclose(got, ref, rtol=2.0 ** -7, atol=1e-6)
+        assert torch.equal(vc[b, :L], v[s0:s0 + L])
+        assert torch.count_nonzero(kc[b, L:]) == 0  # nothing written past the sequence
+
+
+def test_cache_writer_reports_positions_outside_the_cache(jl):
+    cos, sin = _tables(jl, 64, 128, 1e4)
+    q = torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 2, 128), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, 16, 2, 128), dtype=torch.bfloat16, device="cuda")
+    jl.jl_decode_append(q, kv, kv, torch.tensor([40], dtype=torch.int32, device="cuda"), cos, sin, kc, kc.clone())
+    with pytest.raises(jl.JetLongError) as err:
+        jl.jl_sync_status()
+    assert err.value.status == jl.JL_ERR_INVALID
+    jl.jl_sync_status()
+    assert torch.count_nonzero(kc) == 0
+
+
+def test_streaming_decode_from_raw_tokens_across_G_boundary(jl):
+    """Prompt -> jl_kv_cache_fill; then per step jl_decode_append (raw token) + jl_bifocal_decode.
+    Each step must equal the routed attention of the raw sequence's last row (direct definition),
+    across L = 768 -> 769 where G steps from 3 to 4, with no cache rewrite."""
+    L0, steps, w_pre, w0 = 765, 6, 256, 100
+    cfg = I.PrefillConfig("stream", (L0 + steps,), 8, 2, 128, w0, w_pre, 1e4, True)
+    q, k, v, _ = I.prefill_inputs(cfg)
+    stride = L0 + steps
+    cos, sin = _tables(jl, stride, 128, cfg.rope_base)
+    kc = torch.zeros((1, stride, 2, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    cu0 = torch.tensor([0, L0], dtype=torch.int32, device="cuda")
+    jl.jl_kv_cache_fill(k[:L0].cuda(), v[:L0].cuda(), cu0, cos, sin, kc, vc)
+    qb, kb, vb = I.bf16_bits(q), I.bf16_bits(k), I.bf16_bits(v)
+    for t in range(steps):
+        L = L0 + t + 1
+        sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+        qt = jl.jl_decode_append(q[L - 1:L].cuda(), k[L - 1:L].cuda(), v[L - 1:L].cuda(), sl, cos, sin, kc, vc)
+        out, lse = jl.jl_bifocal_decode(qt, kc, vc, sl, stride, w0, w_pre, cos, sin)
+        jl.jl_sync_status()
+        ro, rl = O.bifocal_rows(qb[:L], kb[:L], vb[:L], L, np.full(8, L - 1), np.arange(8), w0=w0,
+                                w_pretrained=w_pre, rope_base=cfg.rope_base)
+        _check(out.float().cpu().numpy()[0], lse.cpu().numpy()[0], ro, rl,
+               f"stream step L={L} G={O.group_size(L, w_pre)}")
