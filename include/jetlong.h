@@ -116,6 +116,28 @@ jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const 
                              const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
                              jl_stream_t stream);
 
+/*
+ * The pages' literal realisation of the bifocal prefill (Methodology section 2):
+ * three flash passes -- pass 1 local window (0 <= i-j < w0) with base
+ * positions, pass 2 full causal with remote positions, pass 3 local window
+ * with remote positions -- each writing its output and log-sum-exp, then the
+ * inclusion-exclusion merge
+ *   M = max(lse1, lse2), a_p = e^(lse_p - M),
+ *   out = (a1 O1 + a2 O2 - a3 O3) / (a1 + a2 - a3), lse = M + ln(a1 + a2 - a3).
+ * Same arguments and result as jl_bifocal_prefill, plus a caller workspace of
+ * jl_bifocal_prefill_three_pass_workspace_size() bytes that afterwards holds
+ * the passes: O_p fp32 [3][total_tokens][Hq][head_dim] (fp32 because the merge
+ * subtracts pass 3 from pass 2), then lse_p fp32 [3][Hq][total_tokens].  It does more work than the fused kernel (pass 3
+ * repeats the window) and exists to run the merge as written.
+ */
+jl_status jl_bifocal_prefill_three_pass(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                        int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq,
+                                        int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
+                                        const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                                        float softmax_scale, void* out, float* lse, void* workspace,
+                                        size_t workspace_bytes, jl_stream_t stream);
+size_t jl_bifocal_prefill_three_pass_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim);
+
 /* Plain causal RoPE prefill (every causal pair LOCAL), built from the same
  * kernel; the comparator for bifocal prefill.  Same conventions. */
 jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,

@@ -101,10 +101,14 @@ jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::
   return ok();
 }
 
-jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+// Validates and fills the kernel parameters; returns JL_OK with *empty set when
+// there is nothing to compute.
+jl_status prefill_params(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                          int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                          int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
-                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, cudaStream_t st) {
+                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, jl::PrefillParams* prm,
+                         bool* empty) {
+  *empty = false;
   if (batch < 0) return fail(JL_ERR_INVALID, "batch must be >= 0 (got %d)", batch);
   if (total_tokens < 0 || total_tokens > 0x7fffffffLL)
     return fail(JL_ERR_INVALID, "total_tokens must be in [0, 2^31) (got %lld)", (long long)total_tokens);
@@ -115,7 +119,10 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
     return fail(JL_ERR_INVALID, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (got Hq=%d, Hkv=%d)", Hq, Hkv);
   if (w0 < 0) return fail(JL_ERR_INVALID, "w0 must be >= 0 (got %d)", w0);
   if (w_pretrained < 1) return fail(JL_ERR_INVALID, "w_pretrained must be >= 1 (got %d)", w_pretrained);
-  if (batch == 0 || total_tokens == 0 || max_seqlen == 0) return ok();
+  if (batch == 0 || total_tokens == 0 || max_seqlen == 0) {
+    *empty = true;
+    return ok();
+  }
   if (!q || !k || !v || !cu_seqlens || !cos_tab || !sin_tab || !out)
     return fail(JL_ERR_INVALID, "null pointer argument");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cos_tab) ||
@@ -123,29 +130,53 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
     return fail(JL_ERR_INVALID, "q, k, v, out and the tables must be 16-byte aligned");
   if (n_tab_rows < max_seqlen)
     return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_seqlen (%d)", (long long)n_tab_rows, max_seqlen);
-  jl::PrefillParams prm{};
-  prm.cu_seqlens = cu_seqlens;
-  prm.cos_tab = cos_tab;
-  prm.sin_tab = sin_tab;
-  prm.out = static_cast<__nv_bfloat16*>(out);
-  prm.lse = lse;
-  prm.total_tokens = total_tokens;
-  prm.n_tab_rows = n_tab_rows;
-  prm.batch = batch;
-  prm.n_qtiles = (max_seqlen + jl::kBM - 1) / jl::kBM;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.group = Hq / Hkv;
-  prm.w0 = w0;
-  prm.w_pre = w_pretrained;
-  prm.plain = plain;
+  *prm = jl::PrefillParams{};
+  prm->cu_seqlens = cu_seqlens;
+  prm->cos_tab = cos_tab;
+  prm->sin_tab = sin_tab;
+  prm->out = static_cast<__nv_bfloat16*>(out);
+  prm->lse = lse;
+  prm->total_tokens = total_tokens;
+  prm->n_tab_rows = n_tab_rows;
+  prm->batch = batch;
+  prm->n_qtiles = (max_seqlen + jl::kBM - 1) / jl::kBM;
+  prm->Hq = Hq;
+  prm->Hkv = Hkv;
+  prm->group = Hq / Hkv;
+  prm->w0 = w0;
+  prm->w_pre = w_pretrained;
+  prm->plain = plain;
+  prm->mode = 0;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
-  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm->scale_log2 = scale * 1.4426950408889634f;
+  prm->slots = prm->group / ((prm->group % 2) == 0 ? 2 : 1);
+  return ok();
+}
+
+jl_status launch_prefill_any(const void* q, const void* k, const void* v, const jl::PrefillParams& prm,
+                             int32_t head_dim, cudaStream_t st) {
   const bool pair = (prm.group % 2) == 0;
-  prm.slots = prm.group / (pair ? 2 : 1);
   if (head_dim == 128)
     return pair ? launch_prefill<128, 2>(q, k, v, prm, st) : launch_prefill<128, 1>(q, k, v, prm, st);
   return pair ? launch_prefill<64, 2>(q, k, v, prm, st) : launch_prefill<64, 1>(q, k, v, prm, st);
+}
+
+jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                         int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                         int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
+                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, cudaStream_t st) {
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
+                               w_pretrained, plain, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
+                               &empty);
+  if (s != JL_OK || empty) return s;
+  return launch_prefill_any(q, k, v, prm, head_dim, st);
+}
+
+size_t three_pass_ws_bytes(int64_t total_tokens, int32_t Hq, int32_t head_dim) {
+  if (total_tokens <= 0 || Hq <= 0 || head_dim <= 0) return 0;
+  return 3 * static_cast<size_t>(total_tokens) * Hq * head_dim * 4 + 3 * static_cast<size_t>(total_tokens) * Hq * 4;
 }
 
 // ------------------------------------------------------------------ decode --
@@ -448,6 +479,48 @@ jl_status jl_decode_append(const void* q, const void* k, const void* v, const in
   else jl::jl_decode_append_kernel<64><<<blocks, 256, 0, st>>>(prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
+  return ok();
+}
+
+size_t jl_bifocal_prefill_three_pass_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim) {
+  return three_pass_ws_bytes(total_tokens, Hq, head_dim);
+}
+
+jl_status jl_bifocal_prefill_three_pass(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                        int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq,
+                                        int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
+                                        const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                                        float softmax_scale, void* out, float* lse, void* workspace,
+                                        size_t workspace_bytes, jl_stream_t stream) {
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
+                               w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm, &empty);
+  if (s != JL_OK || empty) return s;
+  const size_t need = three_pass_ws_bytes(total_tokens, Hq, head_dim);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need)
+    return fail(JL_ERR_INVALID, "three-pass workspace: %zu bytes needed, 16-byte aligned", need);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* o3x = static_cast<float*>(workspace);  // fp32: the merge subtracts pass 3 from pass 2
+  const int64_t plane = total_tokens * Hq * head_dim;
+  float* lse3x = reinterpret_cast<float*>(o3x + 3 * plane);
+  const int modes[3] = {1, 0, 3};  // pass 1: window/base; pass 2: causal/remote (fused with w0 = 0); pass 3
+  for (int pass = 0; pass < 3; ++pass) {
+    jl::PrefillParams pp = prm;
+    pp.mode = modes[pass];
+    if (pass == 1) pp.w0 = 0;
+    pp.out_f32 = o3x + pass * plane;
+    pp.lse = lse3x + pass * total_tokens * Hq;
+    if ((s = launch_prefill_any(q, k, v, pp, head_dim, st)) != JL_OK) return s;
+  }
+  const int64_t rows = total_tokens * Hq;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (head_dim == 128)
+    jl::jl_ie_merge_kernel<128><<<blocks, 256, 0, st>>>(o3x, lse3x, total_tokens, Hq, prm.out, lse);
+  else
+    jl::jl_ie_merge_kernel<64><<<blocks, 256, 0, st>>>(o3x, lse3x, total_tokens, Hq, prm.out, lse);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }
 

@@ -48,6 +48,7 @@ struct PrefillParams {
   const float* cos_tab;
   const float* sin_tab;
   __nv_bfloat16* out;
+  float* out_f32;        // if set, rows are written in fp32 here instead of bf16 to out
   float* lse;
   int64_t total_tokens;
   int64_t n_tab_rows;
@@ -60,6 +61,7 @@ struct PrefillParams {
   int32_t w0;
   int32_t w_pre;
   int32_t plain;
+  int32_t mode;          // 0: fused bifocal / plain; 1: pass 1 alone; 3: pass 3 alone (see TileSchedule)
   float scale_log2;      // softmax scale * log2(e)
 };
 
@@ -93,17 +95,22 @@ struct PrefillBars {
   int abort;
 };
 
-// Which key tiles a query block visits and in which order.
+// Which key tiles a query block visits and in which order.  The fused kernel
+// (visit_remote) visits remote tiles first, then local tiles.  The literal
+// passes 1 and 3 of the inclusion-exclusion merge visit local tiles only (pass 2
+// is the fused kernel with w0 = 0).
 struct TileSchedule {
   int q_lo, q_hi;  // first / last valid query position of the block
   int n_kt;        // key tiles 0 .. n_kt-1 hold causal pairs
-  int R;           // remote tiles: kt in [0, R)   (hold a pair with i - j >= w0)
-  int Lo;          // local tiles:  kt in [Lo, n_kt) (hold a pair with i - j <  w0)
-  int n_virt;      // R + (n_kt - Lo): remote visits first, then local visits
+  int R;           // tiles holding a pair with i - j >= w0: kt in [0, R)
+  int Lo;          // tiles holding a pair with i - j <  w0: kt in [Lo, n_kt)
+  int n_virt;      // number of visits
   int w0;          // effective window (huge when every pair is local)
+  bool visit_remote;
 
-  __device__ void init(int qt, int L, int w0_eff) {
+  __device__ void init(int qt, int L, int w0_eff, bool with_remote) {
     w0 = w0_eff;
+    visit_remote = with_remote;
     q_lo = qt * kBM;
     q_hi = min(q_lo + kBM - 1, L - 1);
     n_kt = q_hi / kBN + 1;
@@ -114,15 +121,20 @@ struct TileSchedule {
       const int x = q_lo - (kBN - 1) - w0;  // local iff kt * 128 > x
       Lo = (x < 0) ? 0 : min(n_kt, x / kBN + 1);
     }
-    n_virt = R + (n_kt - Lo);
+    n_virt = (visit_remote ? R : 0) + (n_kt - Lo);
   }
-  __device__ bool remote(int n) const { return n < R; }
-  __device__ int kt(int n) const { return n < R ? n : Lo + (n - R); }
+  __device__ int R_visits() const { return visit_remote ? R : 0; }
+  __device__ bool remote(int n) const { return n < R_visits(); }
+  __device__ int kt(int n) const { return n < R_visits() ? n : Lo + (n - R_visits()); }
+  // first visit of a Q rotation phase (remote phase, then local phase)
+  __device__ bool phase_start(int n) const { return n == 0 || n == R_visits(); }
+  // last visit using the remote-rotated Q when a local phase follows
+  __device__ bool phase_end(int n) const { return n == R_visits() - 1 && R_visits() < n_virt; }
   // Does visit n need a per-element mask (window edge or causal diagonal)?
   __device__ bool masked(int n) const {
     const int k = kt(n);
     const bool diag = k * kBN + kBN - 1 > q_lo;
-    return diag || (n < R ? (k >= Lo) : (k < R));
+    return diag || (remote(n) ? (k >= Lo) : (k < R));
   }
 };
 
@@ -293,9 +305,27 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
 
   int G = 1;
   if (!p.plain) G = max(1, (L + p.w_pre - 1) / p.w_pre);
-  const int w0_eff = (p.plain || G == 1) ? (1 << 30) : p.w0;
+  // G = 1 (or plain): remote scores equal base scores, every pair runs as local.
+  // The literal passes keep the real window.
+  const int w0_eff = (p.mode == 0 && (p.plain || G == 1)) ? (1 << 30) : p.w0;
   TileSchedule sc;
-  sc.init(qt, L, w0_eff);
+  sc.init(qt, L, w0_eff, p.mode == 0);
+  // Pass 3 rotates its (local-window) visits by the remote positions.
+  const bool local_uses_remote = (p.mode == 3);
+
+  if (sc.n_virt == 0) {  // an empty pass (w0 = 0 for passes 1 and 3): O = 0, lse = -inf
+    for (int r = threadIdx.x; r < kBM * NQT; r += blockDim.x) {
+      const int i = sc.q_lo + (r % kBM), h = h0 + r / kBM;
+      if (i > sc.q_hi) continue;
+      const int64_t row_off = ((static_cast<int64_t>(seq0) + i) * p.Hq + h) * D;
+      for (int c = 0; c < D; ++c) {
+        if (p.out_f32 != nullptr) p.out_f32[row_off + c] = 0.f;
+        else p.out[row_off + c] = __float2bfloat16_rn(0.f);
+      }
+      if (p.lse != nullptr) p.lse[static_cast<int64_t>(h) * p.total_tokens + seq0 + i] = -INFINITY;
+    }
+    return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -346,7 +376,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       int issued_q = 0;
       int issued[kStages] = {0};
       for (int n = 0; n < sc.n_virt && !*abort; ++n) {
-        if (n == 0 || n == sc.R) {
+        if (sc.phase_start(n)) {
           if (n > 0 && !mbar_wait(&bars->q_empty, 0, abort)) break;
           mbar_arrive_expect_tx(&bars->q_full, kTileTx * NQT);
           for (int t = 0; t < NQT; ++t)
@@ -399,7 +429,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       int n = 0;
       bool ok = true;
       for (; n < sc.n_virt && ok; ++n) {
-        if (n == 0 || n == sc.R) {
+        if (sc.phase_start(n)) {
           if (!(ok = mbar_wait(&bars->q_ready, n == 0 ? 0 : 1, abort))) break;
           tc_fence_after();
         }
@@ -422,7 +452,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
           umma_commit(&bars->s_full[1]);
         }
         umma_commit(&bars->k_empty[s]);
-        if (n == sc.R - 1 && sc.R < sc.n_virt) umma_commit(&bars->q_empty);
+        if (sc.phase_end(n)) umma_commit(&bars->q_empty);
         if (!(ok = mbar_wait(&bars->p_ready[0], n & 1, abort))) break;
         tc_fence_after();
         if (!(ok = mbar_wait(&bars->v_full[s], u & 1, abort))) break;
@@ -456,14 +486,14 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     RotFactor<D> step;  // e^{i theta_c}: table row 1
     load_factor<D>(step, p, 1, lane);
     auto key_anchor = [&](int n) {
-      return slice_anchor_row(sc.kt(n) * kBN, rw, sc.remote(n) ? G : 1);
+      return slice_anchor_row(sc.kt(n) * kBN, rw, (sc.remote(n) || local_uses_remote) ? G : 1);
     };
     RotFactor<D> fk_next;
     load_factor<D>(fk_next, p, key_anchor(0), lane);
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
-      const int g = remote ? G : 1;
-      if (n == 0 || n == sc.R) {
+      const int g = (remote || local_uses_remote) ? G : 1;
+      if (sc.phase_start(n)) {
         RotFactor<D> fq;
         load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane);
         if (!mbar_wait(&bars->q_full, n == 0 ? 0 : 1, abort)) break;
@@ -576,13 +606,19 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const int h = h0 + t;
       const bool valid = i <= sc.q_hi;
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = p.out + ((static_cast<int64_t>(seq0) + i) * p.Hq + h) * D;
+      const int64_t row_off = ((static_cast<int64_t>(seq0) + i) * p.Hq + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(t_o + c * 32, o);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        if (valid && p.out_f32 != nullptr) {
+          float4* dst = reinterpret_cast<float4*>(p.out_f32 + row_off + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv, __uint_as_float(o[4 * v4 + 1]) * inv,
+                                  __uint_as_float(o[4 * v4 + 2]) * inv, __uint_as_float(o[4 * v4 + 3]) * inv);
+        } else if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + row_off + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;
@@ -608,6 +644,38 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
   }
+}
+
+// Literal inclusion-exclusion merge of the three passes (natural-log LSEs):
+//   M = max(lse1, lse2); a_p = e^(lse_p - M) (0 for an empty pass);
+//   Z = a1 + a2 - a3;  out = (a1 O1 + a2 O2 - a3 O3) / Z;  lse = M + ln Z.
+// One warp per (token, head) row.
+template <int D>
+__global__ void __launch_bounds__(256) jl_ie_merge_kernel(const float* __restrict__ o3x,
+                                                          const float* __restrict__ lse3x, int64_t T, int Hq,
+                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= T * Hq) return;
+  const int64_t t = row / Hq;
+  const int h = static_cast<int>(row % Hq);
+  const int64_t plane = T * Hq * D;
+  const float l1 = lse3x[static_cast<int64_t>(h) * T + t];
+  const float l2 = lse3x[T * Hq + static_cast<int64_t>(h) * T + t];
+  const float l3 = lse3x[2 * T * Hq + static_cast<int64_t>(h) * T + t];
+  const float M = fmaxf(l1, l2);
+  const float a1 = l1 == -INFINITY ? 0.f : __expf(l1 - M);
+  const float a2 = l2 == -INFINITY ? 0.f : __expf(l2 - M);
+  const float a3 = l3 == -INFINITY ? 0.f : __expf(l3 - M);
+  const float Z = a1 + a2 - a3;
+  const float inv = 1.f / Z;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) {
+    const int64_t c = row * D + lane * (D / 32) + e;
+    const float v = a1 * o3x[c] + a2 * o3x[plane + c] - a3 * o3x[2 * plane + c];
+    out[c] = __float2bfloat16_rn(v * inv);
+  }
+  if (lane == 0 && lse != nullptr) lse[static_cast<int64_t>(h) * T + t] = M + __logf(Z);
 }
 
 }  // namespace jl

@@ -49,6 +49,9 @@ SIGNATURES = {
                                                  _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
     "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
+    "jl_bifocal_prefill_three_pass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
+                                                     _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "jl_bifocal_prefill_three_pass_workspace_size": (_sz, [_i64, _i32, _i32]),
     "jl_kv_cache_fill": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _i64,
                                         _vp]),
     "jl_decode_append": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
@@ -156,6 +159,25 @@ def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrain
                                    w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out),
                                    _ptr(lse), _stream(stream)), "jl_bifocal_prefill")
     return out, lse
+
+
+def jl_bifocal_prefill_three_pass(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, *,
+                                  softmax_scale: float = 0.0, out=None, lse=None, workspace=None,
+                                  want_lse: bool = True, stream=None):
+    """The literal three-pass inclusion-exclusion prefill; returns (out, lse, workspace).
+
+    The workspace holds the passes afterwards: O_p fp32 [3][T][Hq][d], then lse_p fp32 [3][Hq][T]."""
+    T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
+    need = int(_lib.jl_bifocal_prefill_three_pass_workspace_size(T, hq, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    batch = cu_seqlens.shape[0] - 1
+    _check(_lib.jl_bifocal_prefill_three_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen,
+                                              hq, hkv, d, w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0],
+                                              softmax_scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "jl_bifocal_prefill_three_pass")
+    return out, lse, workspace
 
 
 def jl_plain_prefill(q, k, v, cu_seqlens, max_seqlen: int, cos, sin, *, softmax_scale: float = 0.0, out=None,

@@ -368,3 +368,51 @@ def test_streaming_decode_from_raw_tokens_across_G_boundary(jl):
                                 w_pretrained=w_pre, rope_base=cfg.rope_base)
         _check(out.float().cpu().numpy()[0], lse.cpu().numpy()[0], ro, rl,
                f"stream step L={L} G={O.group_size(L, w_pre)}")
+
+
+# ----------------------------------- literal three-pass inclusion-exclusion ----
+
+THREE_PASS = [
+    ("tp_G4_w0_100", (1000,), 8, 2, 128, 100, 256),
+    ("tp_G4_w0_0", (600,), 4, 2, 128, 0, 160),
+    ("tp_G3_w0_128", (700,), 4, 1, 128, 128, 256),
+    ("tp_G1", (300,), 4, 2, 128, 64, 512),
+    ("tp_varlen", (1, 130, 257, 700, 0, 64), 4, 2, 128, 50, 128),
+    ("tp_w0_covers", (400,), 2, 2, 128, 5000, 100),
+    ("tp_d64_group3", (500,), 3, 1, 64, 40, 100),
+]
+
+
+@pytest.mark.parametrize("case", THREE_PASS, ids=[c[0] for c in THREE_PASS])
+def test_three_pass_merge_on_gpu(jl, case):
+    """The pages' own realisation (pass 1 + pass 2 - pass 3 merged on their LSEs) on the GPU:
+    the merged rows and each pass's LSE match the oracle's direct definition and its
+    three-pass statistics."""
+    name, seqlens, hq, hkv, d, w0, w_pre = case
+    cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    cos, sin = _tables(jl, max(cfg.max_seqlen, 1), d, cfg.rope_base)
+    out, lse, ws = jl.jl_bifocal_prefill_three_pass(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), cfg.max_seqlen, w0,
+                                                    w_pre, cos, sin)
+    jl.jl_sync_status()
+    T = cfg.total_tokens
+    out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    plane = T * hq * d
+    lse_p = ws[3 * plane * 4:].view(torch.float32)[:3 * hq * T].cpu().numpy().reshape(3, hq, T)
+    for s in range(len(seqlens)):
+        L = seqlens[s]
+        if L == 0:
+            continue
+        pos = np.repeat(np.arange(L), hq)
+        head = np.tile(np.arange(hq), L)
+        s0 = int(cu[s])
+        qb, kb, vb = I.bf16_bits(q[s0:s0 + L]), I.bf16_bits(k[s0:s0 + L]), I.bf16_bits(v[s0:s0 + L])
+        ro, rl, rp = O.bifocal_rows(qb, kb, vb, L, pos, head, w0=w0, w_pretrained=w_pre, rope_base=cfg.rope_base,
+                                    three_pass=True)
+        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{name} seq {s} merged")
+        for pss in range(3):
+            got = lse_p[pss][head, s0 + pos]
+            ref = rp[:, pss]
+            assert np.array_equal(np.isneginf(got), np.isneginf(ref)), f"{name} pass {pss + 1} emptiness"
+            fin = np.isfinite(ref)
+            assert np.abs(got[fin] - ref[fin]).max(initial=0.0) <= LSE_MAX, f"{name} pass {pss + 1} lse"
