@@ -117,6 +117,34 @@ jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const 
                              jl_stream_t stream);
 
 /*
+ * Chunked prefill against a base-RoPE cache (a prompt processed in pieces, or
+ * a long continuation of a conversation).  Entry b already holds past_lens[b]
+ * keys/values in the caches, and this chunk's n_b = cu_seqlens[b+1] -
+ * cu_seqlens[b] tokens have been appended after them (jl_kv_cache_fill with
+ * past_lens).  Each chunk query at absolute position i = past_lens[b] + r
+ * attends to cached keys j <= i with the bifocal routing of the current length
+ * L = past_lens[b] + n_b (G = max(1, ceil(L / w_pretrained)), Methodology
+ * section 1).  Local keys are used as cached; remote keys get the correction
+ * rotation R(f(j) - j) in shared memory, the query is rotated by R(f(i)) -- the
+ * cache is never rewritten (Methodology section 2).  The result for a chunk
+ * equals the rows past_lens[b] .. L-1 of a full jl_bifocal_prefill over the
+ * first L tokens.
+ *   q            bf16 [total_tokens][Hq][head_dim], the chunks' RAW queries
+ *   cu_seqlens   device int32 [batch + 1] over the chunks; max_seqlen >= every n_b
+ *   past_lens    device int32 [batch]; max_total >= every past_lens[b] + n_b
+ *   k_cache, v_cache  bf16 [batch][cache_stride][Hkv][head_dim], read only
+ *   out, lse     as for jl_bifocal_prefill, over the chunks' packed tokens
+ * Requirements: cache_stride >= max_total, n_tab_rows >= max_total,
+ * batch * cache_stride < 2^31.
+ */
+jl_status jl_bifocal_prefill_chunk(const void* q, const int32_t* cu_seqlens, const int32_t* past_lens, int32_t batch,
+                                   int64_t total_tokens, int32_t max_seqlen, int32_t max_total, const void* k_cache,
+                                   const void* v_cache, int64_t cache_stride, int32_t Hq, int32_t Hkv,
+                                   int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                                   const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out,
+                                   float* lse, jl_stream_t stream);
+
+/*
  * The pages' literal realisation of the bifocal prefill (Methodology section 2):
  * three flash passes -- pass 1 local window (0 <= i-j < w0) with base
  * positions, pass 2 full causal with remote positions, pass 3 local window
@@ -192,17 +220,19 @@ jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cach
  * un-compressed base keys R(j) k_j at their absolute positions and is written
  * once per token; the bifocal decode only reads it).
  *
- * jl_kv_cache_fill: for every prompt token t of packed sequence b (position
- * p = t - cu_seqlens[b]), k_cache[b][p] = R(p) k[t] (fp32 math, rounded to
- * bf16) and v_cache[b][p] = v[t], for every KV head.
+ * jl_kv_cache_fill: for every token t of packed sequence b (position
+ * p = past_lens[b] + t - cu_seqlens[b]), k_cache[b][p] = R(p) k[t] (fp32 math,
+ * rounded to bf16) and v_cache[b][p] = v[t], for every KV head.
  *   k, v        bf16 [total_tokens][Hkv][head_dim], k RAW
  *   cu_seqlens  device int32 [batch + 1] as for jl_bifocal_prefill
+ *   past_lens   device int32 [batch]: tokens already in each entry (a prompt
+ *               continued in chunks); NULL means 0
  *   k_cache, v_cache  bf16 [batch][cache_stride][Hkv][head_dim]
  * A position >= cache_stride or >= n_tab_rows is skipped and reported by
  * jl_sync_status() as JL_ERR_INVALID (the lengths live on the device).
  */
-jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
-                           int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, const int32_t* past_lens,
+                           int32_t batch, int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
                            const float* sin_tab, int64_t n_tab_rows, void* k_cache, void* v_cache,
                            int64_t cache_stride, jl_stream_t stream);
 

@@ -84,8 +84,10 @@ jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::
   CUtensorMap tq, tk, tv;
   jl_status s;
   if ((s = make_map(&tq, q, prm.total_tokens, prm.Hq, D)) != JL_OK) return s;
-  if ((s = make_map(&tk, k, prm.total_tokens, prm.Hkv, D)) != JL_OK) return s;
-  if ((s = make_map(&tv, v, prm.total_tokens, prm.Hkv, D)) != JL_OK) return s;
+  // keys/values: the packed prompt, or (chunked prefill) the base-RoPE caches
+  const int64_t kv_rows = prm.cached ? static_cast<int64_t>(prm.batch) * prm.cache_stride : prm.total_tokens;
+  if ((s = make_map(&tk, k, kv_rows, prm.Hkv, D)) != JL_OK) return s;
+  if ((s = make_map(&tv, v, kv_rows, prm.Hkv, D)) != JL_OK) return s;
   auto kern = jl::jl_prefill_kernel<D, NQT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -412,8 +414,8 @@ jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const in
                         sin_tab, n_tab_rows, softmax_scale, out, lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
-jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
-                           int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, const int32_t* past_lens,
+                           int32_t batch, int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
                            const float* sin_tab, int64_t n_tab_rows, void* k_cache, void* v_cache,
                            int64_t cache_stride, jl_stream_t stream) {
   if (batch < 0 || total_tokens < 0 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1)
@@ -427,6 +429,7 @@ jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqle
   prm.k = static_cast<const __nv_bfloat16*>(k);
   prm.v = static_cast<const __nv_bfloat16*>(v);
   prm.lens = cu_seqlens;
+  prm.past = past_lens;
   prm.cos_tab = cos_tab;
   prm.sin_tab = sin_tab;
   prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
@@ -480,6 +483,33 @@ jl_status jl_decode_append(const void* q, const void* k, const void* v, const in
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
   return ok();
+}
+
+jl_status jl_bifocal_prefill_chunk(const void* q, const int32_t* cu_seqlens, const int32_t* past_lens, int32_t batch,
+                                   int64_t total_tokens, int32_t max_seqlen, int32_t max_total, const void* k_cache,
+                                   const void* v_cache, int64_t cache_stride, int32_t Hq, int32_t Hkv,
+                                   int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
+                                   const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out,
+                                   float* lse, jl_stream_t stream) {
+  if (!past_lens && batch > 0) return fail(JL_ERR_INVALID, "past_lens is required");
+  if (max_total < max_seqlen) return fail(JL_ERR_INVALID, "max_total must be >= max_seqlen");
+  if (cache_stride < max_total)
+    return fail(JL_ERR_INVALID, "cache_stride (%lld) must be >= max_total (%d)", (long long)cache_stride, max_total);
+  if (static_cast<int64_t>(batch) * cache_stride > 0x7fffffffLL)
+    return fail(JL_ERR_UNSUPPORTED, "batch * cache_stride must be < 2^31");
+  if (n_tab_rows < max_total)
+    return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_total (%d)", (long long)n_tab_rows, max_total);
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return fail(JL_ERR_INVALID, "caches must be 16-byte aligned");
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k_cache, v_cache, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim,
+                               w0, w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
+                               &empty);
+  if (s != JL_OK || empty) return s;
+  prm.cached = 1;
+  prm.past_lens = past_lens;
+  prm.cache_stride = cache_stride;
+  return launch_prefill_any(q, k_cache, v_cache, prm, head_dim, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t jl_bifocal_prefill_three_pass_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim) {

@@ -22,6 +22,7 @@ struct AppendParams {
   const __nv_bfloat16* k;      // raw key rows
   const __nv_bfloat16* v;
   const int32_t* lens;         // fill: cu_seqlens [batch+1]; decode: seqlens [B]
+  const int32_t* past;         // fill: tokens already in each cache entry (NULL = 0)
   const float* cos_tab;
   const float* sin_tab;
   __nv_bfloat16* q_out;        // decode: rotated query rows
@@ -56,7 +57,7 @@ __device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, __
   for (int e = 0; e < PER; ++e) y[lane * PER + e] = x[lane * PER + e];
 }
 
-// Prompt tokens: token t of sequence b sits at position t - cu_seqlens[b].
+// Prompt tokens: token t of sequence b sits at position past[b] + t - cu_seqlens[b].
 template <int D>
 __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;  // (token, head)
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
     if (p.lens[mid] <= t) lo = mid; else hi = mid - 1;
   }
   const int b = lo;
-  const int64_t pos = t - p.lens[b];
+  const int64_t pos = t - p.lens[b] + (p.past != nullptr ? p.past[b] : 0);
   if (pos < 0 || pos >= p.cache_stride || pos >= p.n_tab_rows) {
     if (lane == 0) atomicOr(&g_status, kDevErrBounds);
     return;

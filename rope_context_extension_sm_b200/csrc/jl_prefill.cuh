@@ -62,6 +62,9 @@ struct PrefillParams {
   int32_t w_pre;
   int32_t plain;
   int32_t mode;          // 0: fused bifocal / plain; 1: pass 1 alone; 3: pass 3 alone (see TileSchedule)
+  int32_t cached;        // keys/values come from a base-RoPE cache (chunked prefill)
+  const int32_t* past_lens;  // cached: tokens in each cache entry before this chunk
+  int64_t cache_stride;      // cached: positions per cache entry
   float scale_log2;      // softmax scale * log2(e)
 };
 
@@ -108,10 +111,10 @@ struct TileSchedule {
   int w0;          // effective window (huge when every pair is local)
   bool visit_remote;
 
-  __device__ void init(int qt, int L, int w0_eff, bool with_remote) {
+  __device__ void init(int q_first, int L, int w0_eff, bool with_remote) {
     w0 = w0_eff;
     visit_remote = with_remote;
-    q_lo = qt * kBM;
+    q_lo = q_first;
     q_hi = min(q_lo + kBM - 1, L - 1);
     n_kt = q_hi / kBN + 1;
     R = (q_hi >= w0) ? min(n_kt, (q_hi - w0) / kBN + 1) : 0;
@@ -172,9 +175,11 @@ __device__ __forceinline__ void advance(RotFactor<D>& f, const RotFactor<D>& st)
   }
 }
 
-// Rotate row r of a 128-byte-swizzled [128 rows][D] bf16 tile in place with factor f.
-template <int D>
+// Rotate row r of a 128-byte-swizzled [128 rows][D] bf16 tile in place with factor
+// f = (cos, sin)(m theta): by R(m), or by R(-m) when INV.
+template <int D, bool INV = false>
 __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, const RotFactor<D>& f, int lane) {
+  constexpr float sg = INV ? -1.f : 1.f;
   if constexpr (D == 128) {
     // elements 2l, 2l+1 (box 0) and 64+2l, 64+2l+1 (box 1) share the swizzled offset
     const int off = r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + ((lane & 3) << 2);
@@ -182,11 +187,12 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, const RotFactor
     __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
     const float2 a = __bfloat1622float2(*plo);
     const float2 b = __bfloat1622float2(*phi);
+    const float s0 = sg * f.s[0], s1 = sg * f.s[1];
     float2 ya, yb;
-    ya.x = a.x * f.c[0] - b.x * f.s[0];
-    yb.x = b.x * f.c[0] + a.x * f.s[0];
-    ya.y = a.y * f.c[1] - b.y * f.s[1];
-    yb.y = b.y * f.c[1] + a.y * f.s[1];
+    ya.x = a.x * f.c[0] - b.x * s0;
+    yb.x = b.x * f.c[0] + a.x * s0;
+    ya.y = a.y * f.c[1] - b.y * s1;
+    yb.y = b.y * f.c[1] + a.y * s1;
     *plo = __float22bfloat162_rn(ya);
     *phi = __float22bfloat162_rn(yb);
   } else {
@@ -197,8 +203,9 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, const RotFactor
     __nv_bfloat16* pa = reinterpret_cast<__nv_bfloat16*>(tile + off0);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(tile + off1);
     const float a = __bfloat162float(*pa), b = __bfloat162float(*pb);
-    *pa = __float2bfloat16_rn(a * f.c[0] - b * f.s[0]);
-    *pb = __float2bfloat16_rn(b * f.c[0] + a * f.s[0]);
+    const float sn = sg * f.s[0];
+    *pa = __float2bfloat16_rn(a * f.c[0] - b * sn);
+    *pb = __float2bfloat16_rn(b * f.c[0] + a * sn);
   }
 }
 
@@ -214,10 +221,10 @@ __device__ __forceinline__ int64_t slice_anchor_row(int base, int rw, int g) {
 // slice's first row; the remote position advances by one every g rows.
 // Rotate rows [32 rw, 32 rw + 32) of a tile whose row r sits at position base + r:
 // by R(pos) when g == 1, by R(floor(pos / g)) otherwise.  f is the factor of the
-// slice's first row; the (remote) position steps up every g rows.  Tile bases are
-// multiples of 128 and slices start at multiples of 32, so for GS = g in {1, 2, 4}
-// the slice starts on a group boundary and the step rows are known at compile
-// time; GS = 0 handles any g with a running counter and selects.
+// slice's first row; the (remote) position steps up every g rows.  When base is a
+// multiple of 32, slices start on a group boundary for GS = g in {1, 2, 4} and the
+// step rows are known at compile time; GS = 0 handles any g and any base with a
+// running counter and selects.
 template <int D, int GS>
 __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, int g, RotFactor<D> f,
                                              const RotFactor<D>& st, int lane) {
@@ -248,11 +255,47 @@ __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, in
 template <int D>
 __device__ __forceinline__ void rotate_slice_any(uint8_t* tile, int rw, int base, int g, const RotFactor<D>& f,
                                                  const RotFactor<D>& st, int lane) {
+  if ((base & 31) != 0) {  // a chunk's query block need not start on a multiple of 32
+    rotate_slice<D, 0>(tile, rw, base, g, f, st, lane);
+    return;
+  }
   switch (g) {
     case 1: rotate_slice<D, 1>(tile, rw, base, g, f, st, lane); break;
     case 2: rotate_slice<D, 2>(tile, rw, base, g, f, st, lane); break;
     case 4: rotate_slice<D, 4>(tile, rw, base, g, f, st, lane); break;
     default: rotate_slice<D, 0>(tile, rw, base, g, f, st, lane); break;
+  }
+}
+
+// Correct rows [32 rw, 32 rw + 32) of a cached (base-RoPE) key tile at positions
+// kbase + r to their remote rotation: R(f(j) - j) = R(-n_j), n_j = j - floor(j/G).
+// n steps by one per row except where f steps up; kbase is a multiple of 128, so
+// for G in {2, 4} those rows are compile-time.  f holds (cos, sin)(n theta) of the
+// slice's first row.
+template <int D, int GS>
+__device__ __forceinline__ void correct_slice(uint8_t* tile, int rw, int kbase, int G, RotFactor<D> f,
+                                              const RotFactor<D>& st, int lane) {
+  uint8_t* slice = tile + 32 * rw * 128;
+  if constexpr (GS > 0) {
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      rotate_row<D, true>(slice, r, f, lane);
+      if ((r + 1) % GS != 0) advance<D>(f, st);
+    }
+  } else {
+    int cnt = (kbase + 32 * rw) % G;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      rotate_row<D, true>(slice, r, f, lane);
+      cnt = (cnt + 1 == G) ? 0 : cnt + 1;
+      RotFactor<D> nf = f;
+      advance<D>(nf, st);
+#pragma unroll
+      for (int e = 0; e < RotFactor<D>::NF; ++e) {
+        f.c[e] = cnt != 0 ? nf.c[e] : f.c[e];
+        f.s[e] = cnt != 0 ? nf.s[e] : f.s[e];
+      }
+    }
   }
 }
 
@@ -298,10 +341,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   const int b = (rem / p.slots) % p.batch;
   const int slot = rem % p.slots;
   const int h0 = hkv * p.group + slot * NQT;
-  const int seq0 = p.cu_seqlens[b];
-  const int L = p.cu_seqlens[b + 1] - seq0;
-  if (qt * kBM >= L) return;  // uniform across the CTA, before any barrier exists
+  const int seq0 = p.cu_seqlens[b];                 // packed index of the sequence's first query
+  const int n_rows = p.cu_seqlens[b + 1] - seq0;    // queries of this sequence (or chunk)
+  if (qt * kBM >= n_rows) return;  // uniform across the CTA, before any barrier exists
   if (status_failed()) return;
+  const int past = p.cached ? p.past_lens[b] : 0;   // chunked prefill: keys already cached
+  const int L = past + n_rows;                      // sequence length after this chunk
+  const int q_tok0 = seq0 + qt * kBM;               // packed index of the block's first query
 
   int G = 1;
   if (!p.plain) G = max(1, (L + p.w_pre - 1) / p.w_pre);
@@ -309,7 +355,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   // The literal passes keep the real window.
   const int w0_eff = (p.mode == 0 && (p.plain || G == 1)) ? (1 << 30) : p.w0;
   TileSchedule sc;
-  sc.init(qt, L, w0_eff, p.mode == 0);
+  sc.init(past + qt * kBM, L, w0_eff, p.mode == 0);
   // Pass 3 rotates its (local-window) visits by the remote positions.
   const bool local_uses_remote = (p.mode == 3);
 
@@ -317,12 +363,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     for (int r = threadIdx.x; r < kBM * NQT; r += blockDim.x) {
       const int i = sc.q_lo + (r % kBM), h = h0 + r / kBM;
       if (i > sc.q_hi) continue;
-      const int64_t row_off = ((static_cast<int64_t>(seq0) + i) * p.Hq + h) * D;
+      const int64_t tok = q_tok0 + (r % kBM);
+      const int64_t row_off = (tok * p.Hq + h) * D;
       for (int c = 0; c < D; ++c) {
         if (p.out_f32 != nullptr) p.out_f32[row_off + c] = 0.f;
         else p.out[row_off + c] = __float2bfloat16_rn(0.f);
       }
-      if (p.lse != nullptr) p.lse[static_cast<int64_t>(h) * p.total_tokens + seq0 + i] = -INFINITY;
+      if (p.lse != nullptr) p.lse[static_cast<int64_t>(h) * p.total_tokens + tok] = -INFINITY;
     }
     return;
   }
@@ -382,12 +429,12 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
           for (int t = 0; t < NQT; ++t)
             for (int bx = 0; bx < NBOX; ++bx)
               tma_load_3d(sQ + t * Lay::kTileBytes + bx * Lay::kBoxBytes, &tm_q, &bars->q_full, bx * 64, h0 + t,
-                          seq0 + sc.q_lo);
+                          q_tok0);
           ++issued_q;
         }
         const int s = n % kStages;
         const uint32_t u = n / kStages;
-        const int key0 = seq0 + sc.kt(n) * kBN;
+        const int key0 = p.cached ? static_cast<int>(b * p.cache_stride) + sc.kt(n) * kBN : seq0 + sc.kt(n) * kBN;
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         for (int bx = 0; bx < NBOX; ++bx)
@@ -485,7 +532,11 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     const int rw = Lay::rot_index(warp);
     RotFactor<D> step;  // e^{i theta_c}: table row 1
     load_factor<D>(step, p, 1, lane);
-    auto key_anchor = [&](int n) {
+    auto key_anchor = [&](int n) -> int64_t {
+      if (p.cached) {  // correction index n_j = j - f(j) of the slice's first cached key
+        const int j = sc.kt(n) * kBN + 32 * rw;
+        return j - j / G;
+      }
       return slice_anchor_row(sc.kt(n) * kBN, rw, (sc.remote(n) || local_uses_remote) ? G : 1);
     };
     RotFactor<D> fk_next;
@@ -506,7 +557,15 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (n + 1 < sc.n_virt) load_factor<D>(fk_next, p, key_anchor(n + 1), lane);  // prefetch a tile ahead
       const int s = n % kStages;
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
-      rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
+      if (!p.cached) {
+        rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
+      } else if (g > 1) {  // cached keys are base-rotated: local visits use them as they are
+        switch (g) {
+          case 2: correct_slice<D, 2>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane); break;
+          case 4: correct_slice<D, 4>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane); break;
+          default: correct_slice<D, 0>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane); break;
+        }
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);
@@ -606,7 +665,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const int h = h0 + t;
       const bool valid = i <= sc.q_hi;
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      const int64_t row_off = ((static_cast<int64_t>(seq0) + i) * p.Hq + h) * D;
+      const int64_t row_off = ((static_cast<int64_t>(q_tok0) + row) * p.Hq + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -632,7 +691,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       }
       if (valid && p.lse != nullptr) {
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        p.lse[static_cast<int64_t>(h) * p.total_tokens + seq0 + i] = (m_use + log2f(l_run)) * 0.69314718055994531f;
+        p.lse[static_cast<int64_t>(h) * p.total_tokens + q_tok0 + row] = (m_use + log2f(l_run)) * 0.69314718055994531f;
       }
     }
   }

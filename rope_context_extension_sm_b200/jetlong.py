@@ -49,11 +49,13 @@ SIGNATURES = {
                                                  _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
     "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
+    "jl_bifocal_prefill_chunk": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _i32,
+                                                _i32, _i32, _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_prefill_three_pass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
                                                      _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_prefill_three_pass_workspace_size": (_sz, [_i64, _i32, _i32]),
-    "jl_kv_cache_fill": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _i64,
-                                        _vp]),
+    "jl_kv_cache_fill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp,
+                                        _i64, _vp]),
     "jl_decode_append": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
                                         _i64, _vp]),
 }
@@ -161,6 +163,29 @@ def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrain
     return out, lse
 
 
+def jl_bifocal_prefill_chunk(q, cu_seqlens, past_lens, max_seqlen: int, max_total: int, k_cache, v_cache, w0: int,
+                             w_pretrained: int, cos, sin, *, softmax_scale: float = 0.0, out=None, lse=None,
+                             want_lse: bool = True, stream=None):
+    """Chunked bifocal prefill: chunk queries (raw, packed by cu_seqlens) against base-RoPE
+    caches that already hold past_lens[b] tokens plus this chunk.  Returns (out, lse)."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
+    _need(past_lens, torch.int32, "past_lens", 1)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    T, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=q.device)
+    batch = cu_seqlens.shape[0] - 1
+    _check(_lib.jl_bifocal_prefill_chunk(_ptr(q), _ptr(cu_seqlens), _ptr(past_lens), batch, T, max_seqlen, max_total,
+                                         _ptr(k_cache), _ptr(v_cache), k_cache.shape[1], hq, k_cache.shape[2], d, w0,
+                                         w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out),
+                                         _ptr(lse), _stream(stream)), "jl_bifocal_prefill_chunk")
+    return out, lse
+
+
 def jl_bifocal_prefill_three_pass(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, *,
                                   softmax_scale: float = 0.0, out=None, lse=None, workspace=None,
                                   want_lse: bool = True, stream=None):
@@ -191,15 +216,19 @@ def jl_plain_prefill(q, k, v, cu_seqlens, max_seqlen: int, cos, sin, *, softmax_
     return out, lse
 
 
-def jl_kv_cache_fill(k, v, cu_seqlens, cos, sin, k_cache, v_cache, *, stream=None):
-    """Write R(p) k and v of every prompt token into base-RoPE caches [B][stride][Hkv][d]."""
+def jl_kv_cache_fill(k, v, cu_seqlens, cos, sin, k_cache, v_cache, *, past_lens=None, stream=None):
+    """Write R(p) k and v of every token into base-RoPE caches [B][stride][Hkv][d] at
+    positions p = past_lens[b] + (token index within its sequence)."""
+    if past_lens is not None:
+        _need(past_lens, torch.int32, "past_lens", 1)
     _need(k, torch.bfloat16, "k", 3)
     _need(v, torch.bfloat16, "v", 3)
     _need(cu_seqlens, torch.int32, "cu_seqlens", 1)
     _need(k_cache, torch.bfloat16, "k_cache", 4)
     _need(v_cache, torch.bfloat16, "v_cache", 4)
     T, hkv, d = k.shape
-    _check(_lib.jl_kv_cache_fill(_ptr(k), _ptr(v), _ptr(cu_seqlens), cu_seqlens.shape[0] - 1, T, hkv, d, _ptr(cos),
+    _check(_lib.jl_kv_cache_fill(_ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(past_lens), cu_seqlens.shape[0] - 1, T,
+                                 hkv, d, _ptr(cos),
                                  _ptr(sin), cos.shape[0], _ptr(k_cache), _ptr(v_cache), k_cache.shape[1],
                                  _stream(stream)), "jl_kv_cache_fill")
     return k_cache, v_cache

@@ -416,3 +416,61 @@ def test_three_pass_merge_on_gpu(jl, case):
             assert np.array_equal(np.isneginf(got), np.isneginf(ref)), f"{name} pass {pss + 1} emptiness"
             fin = np.isfinite(ref)
             assert np.abs(got[fin] - ref[fin]).max(initial=0.0) <= LSE_MAX, f"{name} pass {pss + 1} lse"
+
+
+# ---------------------------------------------- chunked prefill over a cache ----
+
+def _chunked_run(jl, name, lens_total, chunk_plan, hq, hkv, d, w0, w_pre):
+    """Prefill each sequence in chunks: append the chunk's keys after the cached ones, then
+    attend the chunk's queries over the cache; every chunk row must equal the direct
+    definition over the raw prefix of length L = past + chunk."""
+    B = len(lens_total)
+    cfg = I.PrefillConfig(name, tuple(lens_total), hq, hkv, d, w0, w_pre, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    stride = max(lens_total)
+    cos, sin = _tables(jl, stride, d, cfg.rope_base)
+    kc = torch.zeros((B, stride, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    past = [0] * B
+    for step in chunk_plan:  # step: chunk length per sequence
+        rows_q, rows_k, rows_v, cu_c = [], [], [], [0]
+        for b in range(B):
+            s0 = int(cu[b]) + past[b]
+            rows_q.append(q[s0:s0 + step[b]])
+            rows_k.append(k[s0:s0 + step[b]])
+            rows_v.append(v[s0:s0 + step[b]])
+            cu_c.append(cu_c[-1] + step[b])
+        qc, kk, vv = torch.cat(rows_q), torch.cat(rows_k), torch.cat(rows_v)
+        cu_t = torch.tensor(cu_c, dtype=torch.int32, device="cuda")
+        past_t = torch.tensor(past, dtype=torch.int32, device="cuda")
+        jl.jl_kv_cache_fill(kk.cuda(), vv.cuda(), cu_t, cos, sin, kc, vc, past_lens=past_t)
+        out, lse = jl.jl_bifocal_prefill_chunk(qc.cuda(), cu_t, past_t, max(max(step), 1),
+                                               max(p + s for p, s in zip(past, step)), kc, vc, w0, w_pre, cos, sin)
+        jl.jl_sync_status()
+        out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+        for b in range(B):
+            n = step[b]
+            if n == 0:
+                continue
+            L = past[b] + n
+            s0 = int(cu[b])
+            pos = np.repeat(np.arange(past[b], L), hq)
+            head = np.tile(np.arange(hq), n)
+            ro, rl = O.bifocal_rows(I.bf16_bits(q[s0:s0 + L]), I.bf16_bits(k[s0:s0 + L]), I.bf16_bits(v[s0:s0 + L]),
+                                    L, pos, head, w0=w0, w_pretrained=w_pre, rope_base=cfg.rope_base)
+            r0 = cu_c[b] + (pos - past[b])
+            _check(out[r0, head], lse[head, r0], ro, rl, f"{name} seq {b} chunk past={past[b]} L={L}")
+        past = [p + s for p, s in zip(past, step)]
+
+
+def test_chunked_prefill_single_sequence_across_G(jl):
+    # L after each chunk: 300 (G 2), 777 (G 4), 1100 (G 5); chunk starts not multiples of 128
+    _chunked_run(jl, "chunk1", [1100], [[300], [477], [323]], 8, 2, 128, 100, 256)
+
+
+def test_chunked_prefill_batched_mixed_pasts(jl):
+    _chunked_run(jl, "chunk_b", [700, 260, 513], [[128, 0, 100], [200, 260, 1], [372, 0, 412]], 4, 2, 128, 64, 128)
+
+
+def test_chunked_prefill_d64_group3(jl):
+    _chunked_run(jl, "chunk_d64", [500], [[129], [371]], 3, 1, 64, 40, 100)
