@@ -251,6 +251,32 @@ jl_status jl_decode_append(const void* q, const void* k, const void* v, const in
                            jl_stream_t stream);
 
 /*
+ * Paged caches.  The caches are a pool of pages, bf16 [num_pages][page_size]
+ * [Hkv][head_dim] (k_pool base-RoPE, v_pool values), and entry b's position j
+ * lives in page block_table[b * max_pages + j / page_size] at row
+ * j % page_size.  block_table: device int32 [B][max_pages].  The writers skip
+ * and report (jl_sync_status: JL_ERR_INVALID) a page index outside
+ * [0, num_pages); the decode reads such a page as zeros.  page_size must be a
+ * multiple of 128 for the decode (a 128-key tile never crosses a page).
+ */
+jl_status jl_bifocal_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                                  const int32_t* seqlens, int32_t B, int32_t max_pages, int32_t page_size,
+                                  int32_t num_pages, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                  int32_t w0, int32_t w_pretrained, const float* cos_tab, const float* sin_tab,
+                                  int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, jl_stream_t stream);
+jl_status jl_kv_cache_fill_paged(const void* k, const void* v, const int32_t* cu_seqlens, const int32_t* past_lens,
+                                 int32_t batch, int64_t total_tokens, int32_t Hkv, int32_t head_dim,
+                                 const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, void* k_pool,
+                                 void* v_pool, const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                 int32_t num_pages, jl_stream_t stream);
+jl_status jl_decode_append_paged(const void* q, const void* k, const void* v, const int32_t* seqlens, int32_t B,
+                                 int32_t Hq, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+                                 const float* sin_tab, int64_t n_tab_rows, void* q_out, void* k_pool, void* v_pool,
+                                 const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                 int32_t num_pages, jl_stream_t stream);
+
+/*
  * jl_bifocal_decode without a caller workspace.  The paper has no counterpart:
  * this entry point exists for callers that cannot allocate device memory, for
  * example an engine plugin that is handed only its input and output buffers,

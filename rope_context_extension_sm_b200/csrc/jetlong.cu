@@ -213,7 +213,8 @@ jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) 
   using Lay = jl::DecTcLayout<GROUP>;
   CUtensorMap tk, tv;
   jl_status s;
-  const int64_t rows = static_cast<int64_t>(B) * prm.cache_stride;
+  // contiguous caches, or (paged) the page pool; the kernel bounds every page it reads
+  const int64_t rows = prm.block_table != nullptr ? prm.cache_stride : static_cast<int64_t>(B) * prm.cache_stride;
   if ((s = make_map(&tk, prm.k, rows, prm.Hkv, 128)) != JL_OK) return s;
   if ((s = make_map(&tv, prm.v, rows, prm.Hkv, 128)) != JL_OK) return s;
   auto kern = jl::jl_decode_tc_kernel<GROUP, PLAIN>;
@@ -286,7 +287,8 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
                         int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                         int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
-                        size_t workspace_bytes, cudaStream_t st) {
+                        size_t workspace_bytes, cudaStream_t st, const int32_t* block_table = nullptr,
+                        int32_t page_size = 0, int32_t max_pages = 0) {
   if (B < 0) return fail(JL_ERR_INVALID, "B must be >= 0 (got %d)", B);
   if (head_dim != 64 && head_dim != 128)
     return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
@@ -301,7 +303,7 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
                 max_seqlen);
   if (n_tab_rows < max_seqlen)
     return fail(JL_ERR_INVALID, "n_tab_rows (%lld) must be >= max_seqlen (%d)", (long long)n_tab_rows, max_seqlen);
-  if (static_cast<int64_t>(B) * cache_stride > 0x7fffffffLL)
+  if (block_table == nullptr && static_cast<int64_t>(B) * cache_stride > 0x7fffffffLL)
     return fail(JL_ERR_UNSUPPORTED, "B * cache_stride must be < 2^31 (got %lld)", (long long)B * cache_stride);
   if (!q || !k_cache || !v_cache || !seqlens || !cos_tab || !sin_tab || !out || !workspace)
     return fail(JL_ERR_INVALID, "null pointer argument");
@@ -321,8 +323,11 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
   prm.ws = static_cast<float*>(workspace);
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
-  prm.cache_stride = cache_stride;
+  prm.cache_stride = cache_stride;  // paged: rows of the page pool
   prm.n_tab_rows = n_tab_rows;
+  prm.block_table = block_table;
+  prm.page_size = page_size;
+  prm.max_pages = max_pages;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
@@ -336,6 +341,57 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
   if (head_dim == 128)
     return plain ? dispatch_group<128, true>(prm, B, st) : dispatch_group<128, false>(prm, B, st);
   return plain ? dispatch_group<64, true>(prm, B, st) : dispatch_group<64, false>(prm, B, st);
+}
+
+// ------------------------------------------------------------ cache writers --
+
+// fill = true: prompt tokens (packed by lens = cu_seqlens, optional past offsets);
+// fill = false: one decode token per entry (lens = seqlens), query rotated to q_out.
+jl_status append_common(const void* q, const void* k, const void* v, const int32_t* lens, const int32_t* past,
+                        int32_t batch, int64_t total_tokens, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                        const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, void* q_out, void* k_cache,
+                        void* v_cache, int64_t cache_stride, const int32_t* block_table, int32_t page_size,
+                        int32_t max_pages, int32_t num_pages, cudaStream_t st, bool fill) {
+  if (batch < 0 || total_tokens < 0 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1 || (!fill && Hq < 1))
+    return fail(JL_ERR_INVALID, "need batch >= 0, tokens >= 0, heads >= 1, cache_stride >= 1, n_tab_rows >= 1");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (batch == 0 || (fill && total_tokens == 0)) return ok();
+  if (!k || !v || !lens || !cos_tab || !sin_tab || !k_cache || !v_cache || (!fill && (!q || !q_out)))
+    return fail(JL_ERR_INVALID, "null pointer argument");
+  jl::AppendParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k);
+  prm.v = static_cast<const __nv_bfloat16*>(v);
+  prm.lens = lens;
+  prm.past = past;
+  prm.cos_tab = cos_tab;
+  prm.sin_tab = sin_tab;
+  prm.q_out = static_cast<__nv_bfloat16*>(q_out);
+  prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  prm.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  prm.total_tokens = total_tokens;
+  prm.cache_stride = cache_stride;  // paged: positions one entry can hold (max_pages * page_size)
+  prm.n_tab_rows = n_tab_rows;
+  prm.batch = batch;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.block_table = block_table;
+  prm.page_size = page_size;
+  prm.max_pages = max_pages;
+  prm.num_pages = num_pages;
+  const int64_t rows = fill ? total_tokens * Hkv : static_cast<int64_t>(batch) * (Hq + Hkv);
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  if (fill) {
+    if (head_dim == 128) jl::jl_kv_fill_kernel<128><<<blocks, 256, 0, st>>>(prm);
+    else jl::jl_kv_fill_kernel<64><<<blocks, 256, 0, st>>>(prm);
+  } else {
+    if (head_dim == 128) jl::jl_decode_append_kernel<128><<<blocks, 256, 0, st>>>(prm);
+    else jl::jl_decode_append_kernel<64><<<blocks, 256, 0, st>>>(prm);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, fill ? "kv fill launch" : "decode append launch");
+  return ok();
 }
 
 }  // namespace
@@ -418,71 +474,43 @@ jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqle
                            int32_t batch, int64_t total_tokens, int32_t Hkv, int32_t head_dim, const float* cos_tab,
                            const float* sin_tab, int64_t n_tab_rows, void* k_cache, void* v_cache,
                            int64_t cache_stride, jl_stream_t stream) {
-  if (batch < 0 || total_tokens < 0 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1)
-    return fail(JL_ERR_INVALID, "need batch >= 0, total_tokens >= 0, Hkv >= 1, cache_stride >= 1, n_tab_rows >= 1");
-  if (head_dim != 64 && head_dim != 128)
-    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
-  if (batch == 0 || total_tokens == 0) return ok();
-  if (!k || !v || !cu_seqlens || !cos_tab || !sin_tab || !k_cache || !v_cache)
-    return fail(JL_ERR_INVALID, "null pointer argument");
-  jl::AppendParams prm{};
-  prm.k = static_cast<const __nv_bfloat16*>(k);
-  prm.v = static_cast<const __nv_bfloat16*>(v);
-  prm.lens = cu_seqlens;
-  prm.past = past_lens;
-  prm.cos_tab = cos_tab;
-  prm.sin_tab = sin_tab;
-  prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  prm.v_cache = static_cast<__nv_bfloat16*>(v_cache);
-  prm.total_tokens = total_tokens;
-  prm.cache_stride = cache_stride;
-  prm.n_tab_rows = n_tab_rows;
-  prm.batch = batch;
-  prm.Hkv = Hkv;
-  const int64_t rows = total_tokens * Hkv;
-  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 128) jl::jl_kv_fill_kernel<128><<<blocks, 256, 0, st>>>(prm);
-  else jl::jl_kv_fill_kernel<64><<<blocks, 256, 0, st>>>(prm);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "kv fill launch");
-  return ok();
+  return append_common(nullptr, k, v, cu_seqlens, past_lens, batch, total_tokens, 0, Hkv, head_dim, cos_tab,
+                       sin_tab, n_tab_rows, nullptr, k_cache, v_cache, cache_stride, nullptr, 0, 0, 0,
+                       reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+jl_status jl_kv_cache_fill_paged(const void* k, const void* v, const int32_t* cu_seqlens, const int32_t* past_lens,
+                                 int32_t batch, int64_t total_tokens, int32_t Hkv, int32_t head_dim,
+                                 const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, void* k_pool,
+                                 void* v_pool, const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                 int32_t num_pages, jl_stream_t stream) {
+  if (page_size < 1 || max_pages < 1 || num_pages < 1)
+    return fail(JL_ERR_INVALID, "page_size, max_pages and num_pages must be >= 1");
+  if (batch > 0 && !block_table) return fail(JL_ERR_INVALID, "null block_table");
+  return append_common(nullptr, k, v, cu_seqlens, past_lens, batch, total_tokens, 0, Hkv, head_dim, cos_tab,
+                       sin_tab, n_tab_rows, nullptr, k_pool, v_pool, static_cast<int64_t>(max_pages) * page_size,
+                       block_table, page_size, max_pages, num_pages, reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+jl_status jl_decode_append_paged(const void* q, const void* k, const void* v, const int32_t* seqlens, int32_t B,
+                                 int32_t Hq, int32_t Hkv, int32_t head_dim, const float* cos_tab,
+                                 const float* sin_tab, int64_t n_tab_rows, void* q_out, void* k_pool, void* v_pool,
+                                 const int32_t* block_table, int32_t max_pages, int32_t page_size,
+                                 int32_t num_pages, jl_stream_t stream) {
+  if (page_size < 1 || max_pages < 1 || num_pages < 1)
+    return fail(JL_ERR_INVALID, "page_size, max_pages and num_pages must be >= 1");
+  if (B > 0 && !block_table) return fail(JL_ERR_INVALID, "null block_table");
+  return append_common(q, k, v, seqlens, nullptr, B, 0, Hq, Hkv, head_dim, cos_tab, sin_tab, n_tab_rows, q_out,
+                       k_pool, v_pool, static_cast<int64_t>(max_pages) * page_size, block_table, page_size,
+                       max_pages, num_pages, reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 jl_status jl_decode_append(const void* q, const void* k, const void* v, const int32_t* seqlens, int32_t B,
                            int32_t Hq, int32_t Hkv, int32_t head_dim, const float* cos_tab, const float* sin_tab,
                            int64_t n_tab_rows, void* q_out, void* k_cache, void* v_cache, int64_t cache_stride,
                            jl_stream_t stream) {
-  if (B < 0 || Hq < 1 || Hkv < 1 || cache_stride < 1 || n_tab_rows < 1)
-    return fail(JL_ERR_INVALID, "need B >= 0, Hq >= 1, Hkv >= 1, cache_stride >= 1, n_tab_rows >= 1");
-  if (head_dim != 64 && head_dim != 128)
-    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
-  if (B == 0) return ok();
-  if (!q || !k || !v || !seqlens || !cos_tab || !sin_tab || !q_out || !k_cache || !v_cache)
-    return fail(JL_ERR_INVALID, "null pointer argument");
-  jl::AppendParams prm{};
-  prm.q = static_cast<const __nv_bfloat16*>(q);
-  prm.k = static_cast<const __nv_bfloat16*>(k);
-  prm.v = static_cast<const __nv_bfloat16*>(v);
-  prm.lens = seqlens;
-  prm.cos_tab = cos_tab;
-  prm.sin_tab = sin_tab;
-  prm.q_out = static_cast<__nv_bfloat16*>(q_out);
-  prm.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  prm.v_cache = static_cast<__nv_bfloat16*>(v_cache);
-  prm.cache_stride = cache_stride;
-  prm.n_tab_rows = n_tab_rows;
-  prm.batch = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  const int64_t rows = static_cast<int64_t>(B) * (Hq + Hkv);
-  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 128) jl::jl_decode_append_kernel<128><<<blocks, 256, 0, st>>>(prm);
-  else jl::jl_decode_append_kernel<64><<<blocks, 256, 0, st>>>(prm);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
-  return ok();
+  return append_common(q, k, v, seqlens, nullptr, B, 0, Hq, Hkv, head_dim, cos_tab, sin_tab, n_tab_rows, q_out,
+                       k_cache, v_cache, cache_stride, nullptr, 0, 0, 0, reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 jl_status jl_bifocal_prefill_chunk(const void* q, const int32_t* cu_seqlens, const int32_t* past_lens, int32_t batch,
@@ -552,6 +580,28 @@ jl_status jl_bifocal_prefill_three_pass(const void* q, const void* k, const void
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
+}
+
+jl_status jl_bifocal_decode_paged(const void* q, const void* k_pool, const void* v_pool, const int32_t* block_table,
+                                  const int32_t* seqlens, int32_t B, int32_t max_pages, int32_t page_size,
+                                  int32_t num_pages, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                  int32_t w0, int32_t w_pretrained, const float* cos_tab, const float* sin_tab,
+                                  int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, jl_stream_t stream) {
+  if (!decode_uses_tc(head_dim, Hq, Hkv < 1 ? 1 : Hkv) || Hkv < 1)
+    return fail(JL_ERR_UNSUPPORTED, "paged decode needs head_dim 128 and Hq/Hkv <= 16");
+  if (page_size < 128 || page_size % 128 != 0)
+    return fail(JL_ERR_UNSUPPORTED, "page_size must be a positive multiple of 128 (got %d)", page_size);
+  if (max_pages < 1 || static_cast<int64_t>(max_pages) * page_size < max_seqlen)
+    return fail(JL_ERR_INVALID, "max_pages * page_size must cover max_seqlen");
+  if (num_pages < 1 || static_cast<int64_t>(num_pages) * page_size > 0x7fffffffLL)
+    return fail(JL_ERR_INVALID, "num_pages * page_size must be in [1, 2^31)");
+  if (B > 0 && !block_table) return fail(JL_ERR_INVALID, "null block_table");
+  // validated by the contiguous path with the pool as the cache rows, read through the block table
+  return decode_common(q, k_pool, v_pool, seqlens, B, static_cast<int64_t>(num_pages) * page_size, max_seqlen, Hq,
+                       Hkv, head_dim, w0, w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse,
+                       workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), block_table, page_size,
+                       max_pages);
 }
 
 size_t jl_bifocal_decode_workspace_size(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {

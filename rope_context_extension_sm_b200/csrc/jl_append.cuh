@@ -32,7 +32,18 @@ struct AppendParams {
   int64_t cache_stride;
   int64_t n_tab_rows;
   int32_t batch, Hq, Hkv;
+  const int32_t* block_table;  // paged caches (NULL: contiguous [batch][cache_stride])
+  int32_t page_size, max_pages, num_pages;
 };
+
+// Cache row of entry b's position pos (already checked against cache_stride):
+// contiguous, or through the block table; -1 when the page index is outside the pool.
+__device__ __forceinline__ int64_t cache_row(const AppendParams& p, int b, int64_t pos) {
+  if (p.block_table == nullptr) return static_cast<int64_t>(b) * p.cache_stride + pos;
+  const int32_t page = p.block_table[static_cast<int64_t>(b) * p.max_pages + pos / p.page_size];
+  if (page < 0 || page >= p.num_pages) return -1;
+  return static_cast<int64_t>(page) * p.page_size + pos % p.page_size;
+}
 
 // y = R(pos) x for one D-wide bf16 row, lane-parallel; writes y (and copies v_src -> v_dst if given).
 template <int D>
@@ -77,7 +88,12 @@ __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
     return;
   }
   const int64_t src = (t * p.Hkv + h) * D;
-  const int64_t dst = ((static_cast<int64_t>(b) * p.cache_stride + pos) * p.Hkv + h) * D;
+  const int64_t crow = cache_row(p, b, pos);
+  if (crow < 0) {
+    if (lane == 0) atomicOr(&g_status, kDevErrBounds);
+    return;
+  }
+  const int64_t dst = (crow * p.Hkv + h) * D;
   rotate_row_global<D>(p.k + src, p.k_cache + dst, pos, p, lane);
   copy_row<D>(p.v + src, p.v_cache + dst, lane);
 }
@@ -102,7 +118,12 @@ __global__ void __launch_bounds__(256) jl_decode_append_kernel(const AppendParam
   } else {
     const int h = r - p.Hq;
     const int64_t src = (static_cast<int64_t>(b) * p.Hkv + h) * D;
-    const int64_t dst = ((static_cast<int64_t>(b) * p.cache_stride + i) * p.Hkv + h) * D;
+    const int64_t crow = cache_row(p, b, i);
+    if (crow < 0) {
+      if (lane == 0) atomicOr(&g_status, kDevErrBounds);
+      return;
+    }
+    const int64_t dst = (crow * p.Hkv + h) * D;
     rotate_row_global<D>(p.k + src, p.k_cache + dst, i, p, lane);
     copy_row<D>(p.v + src, p.v_cache + dst, lane);
   }

@@ -38,6 +38,8 @@ struct DecodeParams {
   float* lse;
   int64_t cache_stride;   // positions per batch entry
   int64_t n_tab_rows;     // rows of cos_tab / sin_tab
+  const int32_t* block_table;  // paged caches: page of entry b's position j is block_table[b * max_pages + j / page_size]
+  int32_t page_size, max_pages;
   int32_t Hq, Hkv, group;
   int32_t w0, w_pre, plain;
   int32_t chunk, n_split;

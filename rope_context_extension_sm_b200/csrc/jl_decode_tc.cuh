@@ -7,7 +7,9 @@
 // <R(f(i) - i) q~, R(f(j) - j) k~_j> = <R(f(i)) q, R(f(j)) k_j>; local keys score
 // <q~, k~_j>.
 //
-// CTA = (KV head, chunk of keys, batch entry).  Per 128-key tile:
+// CTA = (KV head, chunk of keys, batch entry).  The caches are contiguous per
+// entry, or a page pool with a block table (pages of a multiple of 128 keys, so a
+// tile lies in one page).  Per 128-key tile:
 //   warp 0      TMA producer: raw K and V tiles (3 stages)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-3,  correction warps (16, or 8 for 16 heads per KV head): rotate
@@ -211,7 +213,11 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       for (int n = 0; n < n_tiles && !*abort; ++n) {
         const int s = n % kDecStages;
         const uint32_t u = n / kDecStages;
-        const int key0 = static_cast<int>(row0) + c0 + n * kDecTile;
+        const int kpos = c0 + n * kDecTile;  // key position in entry b; a tile never crosses a page
+        const int key0 = p.block_table != nullptr
+                             ? p.block_table[static_cast<int64_t>(b) * p.max_pages + kpos / p.page_size] * p.page_size +
+                                   kpos % p.page_size
+                             : static_cast<int>(row0) + kpos;
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         tma_load_3d(sK + s * Lay::kTile, &tm_k, &bars->k_full[s], 0, hk, key0);

@@ -49,6 +49,12 @@ SIGNATURES = {
                                                  _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_decode_noalloc_scratch_bytes": (_sz, []),
     "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
+    "jl_bifocal_decode_paged": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                               _i32, _i32, _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "jl_kv_cache_fill_paged": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp,
+                                              _vp, _i32, _i32, _i32, _vp]),
+    "jl_decode_append_paged": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _vp, _vp,
+                                              _vp, _vp, _i32, _i32, _i32, _vp]),
     "jl_bifocal_prefill_chunk": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _i32,
                                                 _i32, _i32, _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
     "jl_bifocal_prefill_three_pass": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
@@ -299,6 +305,53 @@ def jl_plain_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, cos, sin, *, 
                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "jl_plain_decode")
     return out, lse
+
+
+def jl_bifocal_decode_paged(q, k_pool, v_pool, block_table, seqlens, max_seqlen: int, w0: int, w_pretrained: int,
+                            cos, sin, *, softmax_scale: float = 0.0, out=None, lse=None, workspace=None,
+                            want_lse: bool = True, stream=None):
+    """Bifocal decode over paged caches: pools [num_pages][page_size][Hkv][d], block_table [B][max_pages]."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k_pool, torch.bfloat16, "k_pool", 4)
+    _need(v_pool, torch.bfloat16, "v_pool", 4)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seqlens, torch.int32, "seqlens", 1)
+    B, hq, d = q.shape
+    num_pages, page_size, hkv, _ = k_pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    need = jl_bifocal_decode_workspace_size(B, hq, d, max_seqlen)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(_lib.jl_bifocal_decode_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(seqlens), B,
+                                        block_table.shape[1], page_size, num_pages, max_seqlen, hq, hkv, d, w0,
+                                        w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out),
+                                        _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "jl_bifocal_decode_paged")
+    return out, lse
+
+
+def jl_kv_cache_fill_paged(k, v, cu_seqlens, cos, sin, k_pool, v_pool, block_table, *, past_lens=None, stream=None):
+    """jl_kv_cache_fill into paged pools through a block table."""
+    T, hkv, d = k.shape
+    _check(_lib.jl_kv_cache_fill_paged(_ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(past_lens), cu_seqlens.shape[0] - 1,
+                                       T, hkv, d, _ptr(cos), _ptr(sin), cos.shape[0], _ptr(k_pool), _ptr(v_pool),
+                                       _ptr(block_table), block_table.shape[1], k_pool.shape[1], k_pool.shape[0],
+                                       _stream(stream)), "jl_kv_cache_fill_paged")
+
+
+def jl_decode_append_paged(q, k, v, seqlens, cos, sin, k_pool, v_pool, block_table, *, q_out=None, stream=None):
+    """jl_decode_append into paged pools through a block table; returns q~."""
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    B, hq, d = q.shape
+    _check(_lib.jl_decode_append_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), B, hq, k.shape[1], d, _ptr(cos),
+                                       _ptr(sin), cos.shape[0], _ptr(q_out), _ptr(k_pool), _ptr(v_pool),
+                                       _ptr(block_table), block_table.shape[1], k_pool.shape[1], k_pool.shape[0],
+                                       _stream(stream)), "jl_decode_append_paged")
+    return q_out
 
 
 def jl_bifocal_decode_noalloc_scratch_bytes() -> int:

@@ -474,3 +474,80 @@ def test_chunked_prefill_batched_mixed_pasts(jl):
 
 def test_chunked_prefill_d64_group3(jl):
     _chunked_run(jl, "chunk_d64", [500], [[129], [371]], 3, 1, 64, 40, 100)
+
+
+# --------------------------------------------------------------- paged caches ----
+
+def _paginate(cache, lens, page_size, seed=3):
+    """Scatter contiguous caches [B][stride][Hkv][d] into a shuffled page pool + block table."""
+    B = cache.shape[0]
+    max_pages = max(-(-L // page_size) for L in lens)
+    n_pages = sum(-(-L // page_size) for L in lens) + 3
+    order = np.random.default_rng(seed).permutation(n_pages)
+    pool = torch.zeros((n_pages, page_size) + tuple(cache.shape[2:]), dtype=cache.dtype)
+    table = torch.zeros((B, max_pages), dtype=torch.int32)
+    nxt = 0
+    for b, L in enumerate(lens):
+        for pg in range(-(-L // page_size)):
+            page = int(order[nxt])
+            nxt += 1
+            table[b, pg] = page
+            rows = cache[b, pg * page_size:min(L, (pg + 1) * page_size)]
+            pool[page, :rows.shape[0]] = rows
+    return pool, table
+
+
+def test_paged_decode_equals_contiguous_and_oracle(jl):
+    cfg = SMALL_DECODE
+    lens, page = [1000, 300], 256
+    max_len = 1024
+    k_cache, v = _decode_setup(cfg, max_len, batch=2)
+    qs = I.decode_queries(cfg, 1, batch=2)[0]
+    q_t = torch.stack([_query_tilde(cfg, qs[b], lens[b]) for b in range(2)])
+    cos, sin = _tables(jl, max_len, 128, cfg.rope_base)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ref, ref_lse = jl.jl_bifocal_decode(q_t.cuda(), k_cache.cuda(), v.cuda(), sl, max_len, cfg.w0, cfg.w_pretrained,
+                                        cos, sin)
+    kp, table = _paginate(k_cache, lens, page)
+    vp, _ = _paginate(v, lens, page)
+    out, lse = jl.jl_bifocal_decode_paged(q_t.cuda(), kp.cuda(), vp.cuda(), table.cuda(), sl, max_len, cfg.w0,
+                                          cfg.w_pretrained, cos, sin)
+    jl.jl_sync_status()
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+    for b, L in enumerate(lens):
+        ro, rl = _decode_oracle(cfg, q_t[b], k_cache[b], v[b], L)
+        _check(out[b].float().cpu().numpy(), lse[b].cpu().numpy(), ro, rl, f"paged b={b}")
+
+
+def test_paged_cache_writers_match_contiguous(jl):
+    cfg = I.PrefillConfig("pfill", (500, 130), 4, 2, 128, 32, 64, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    cos, sin = _tables(jl, 1024, 128, cfg.rope_base)
+    kc = torch.zeros((2, 512, 2, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    jl.jl_kv_cache_fill(k.cuda(), v.cuda(), cu.cuda(), cos, sin, kc, vc)
+    _, table = _paginate(kc.cpu(), [512, 512], 128)
+    n_pages = int(table.max()) + 1
+    kp = torch.zeros((n_pages, 128, 2, 128), dtype=torch.bfloat16, device="cuda")
+    vp = torch.zeros_like(kp)
+    tb = table.cuda()
+    jl.jl_kv_cache_fill_paged(k.cuda(), v.cuda(), cu.cuda(), cos, sin, kp, vp, tb)
+    # one decode-step append at position 500 of entry 0 and 130 of entry 1
+    q1 = torch.randn((2, 4, 128)).to(torch.bfloat16).cuda()
+    k1 = torch.randn((2, 2, 128)).to(torch.bfloat16).cuda()
+    sl = torch.tensor([501, 131], dtype=torch.int32, device="cuda")
+    qa = jl.jl_decode_append(q1, k1, k1, sl, cos, sin, kc, vc)
+    qb = jl.jl_decode_append_paged(q1, k1, k1, sl, cos, sin, kp, vp, tb)
+    jl.jl_sync_status()
+    assert torch.equal(qa, qb)
+    for b, L in enumerate([501, 131]):
+        for pos in range(L):
+            page, off = int(table[b, pos // 128]), pos % 128
+            assert torch.equal(kp[page, off], kc[b, pos]) and torch.equal(vp[page, off], vc[b, pos])
+    bad = tb.clone()
+    bad[0, 0] = n_pages + 7
+    jl.jl_kv_cache_fill_paged(k.cuda(), v.cuda(), cu.cuda(), cos, sin, kp, vp, bad)
+    with pytest.raises(jl.JetLongError) as err:
+        jl.jl_sync_status()
+    assert err.value.status == jl.JL_ERR_INVALID
+    jl.jl_sync_status()
