@@ -293,6 +293,85 @@ int jlo_bifocal_rows_three_pass(jlo_view q, jlo_view k, jlo_view v, int64_t L, i
                    rope_base, scale, 0, 1, out, lse, pass_lse);
 }
 
+/* ---- frequency-interpolation variant (Results, ablation: aliasing vs interpolation) ---- */
+
+int jlo_interp_rows(jlo_view q, jlo_view k, jlo_view v, int64_t L, int32_t d, int32_t hq, int32_t hkv,
+                    const int64_t* row_pos, const int32_t* row_head, int64_t n_rows, int64_t w0, double base,
+                    const double* lambda, double scale, double* out, double* lse) {
+  if (check_common(L, d, hq, hkv, w0, 1) || !lambda) return -1;
+  int64_t imax = -1;
+  for (int64_t r = 0; r < n_rows; ++r) {
+    if (row_pos[r] < 0 || row_pos[r] >= L || row_head[r] < 0 || row_head[r] >= hq) return -2;
+    if (row_pos[r] > imax) imax = row_pos[r];
+  }
+  if (n_rows == 0) return 0;
+  const int32_t h = d / 2;
+  const int64_t npos = imax + 1;
+  const int32_t group = hq / hkv;
+  double* theta = (double*)malloc(sizeof(double) * (size_t)h);
+  double* cb = (double*)malloc(sizeof(double) * (size_t)(npos * h));  /* base cos/sin */
+  double* sb = (double*)malloc(sizeof(double) * (size_t)(npos * h));
+  double* ci = (double*)malloc(sizeof(double) * (size_t)(npos * h));  /* interpolated cos/sin */
+  double* si = (double*)malloc(sizeof(double) * (size_t)(npos * h));
+  double* kb = (double*)malloc(sizeof(double) * (size_t)(npos * d));
+  double* ki = (double*)malloc(sizeof(double) * (size_t)(npos * d));
+  if (!theta || !cb || !sb || !ci || !si || !kb || !ki) {
+    free(theta); free(cb); free(sb); free(ci); free(si); free(kb); free(ki);
+    return -3;
+  }
+  jlo_inv_freq(d, base, theta);
+#pragma omp parallel for schedule(static)
+  for (int64_t p = 0; p < npos; ++p)
+    for (int32_t c = 0; c < h; ++c) {
+      cb[p * h + c] = cos((double)p * theta[c]);
+      sb[p * h + c] = sin((double)p * theta[c]);
+      ci[p * h + c] = cos((double)p * theta[c] * lambda[c]);
+      si[p * h + c] = sin((double)p * theta[c] * lambda[c]);
+    }
+  for (int32_t kvh = 0; kvh < hkv; ++kvh) {
+    int any = 0;
+    for (int64_t r = 0; r < n_rows && !any; ++r) any = (row_head[r] / group == kvh);
+    if (!any) continue;
+#pragma omp parallel
+    {
+      double* x = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+      for (int64_t j = 0; j < npos; ++j) {
+        view_row(&k, j, kvh, d, x);
+        rotate_with(x, d, cb + j * h, sb + j * h, 1.0, kb + j * d);
+        rotate_with(x, d, ci + j * h, si + j * h, 1.0, ki + j * d);
+      }
+      free(x);
+    }
+#pragma omp parallel
+    {
+      double* x = (double*)malloc(sizeof(double) * (size_t)d * 3);
+      double* qb = x + d;
+      double* qi = qb + d;
+      double* s = (double*)malloc(sizeof(double) * (size_t)npos);
+      unsigned char* mask = (unsigned char*)malloc((size_t)npos);
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t r = 0; r < n_rows; ++r) {
+        if (row_head[r] / group != kvh) continue;
+        const int64_t i = row_pos[r];
+        view_row(&q, i, row_head[r], d, x);
+        rotate_with(x, d, cb + i * h, sb + i * h, 1.0, qb);
+        rotate_with(x, d, ci + i * h, si + i * h, 1.0, qi);
+        for (int64_t j = 0; j < npos; ++j) {
+          const int64_t dist = i - j;
+          if (dist < 0) { mask[j] = MASKED; s[j] = 0.0; }
+          else if (dist < w0) { mask[j] = LOCAL; s[j] = scale * dot(qb, kb + j * d, d); }
+          else { mask[j] = REMOTE; s[j] = scale * dot(qi, ki + j * d, d); }
+        }
+        softmax_row(s, mask, npos, &v, kvh, d, out + r * d, lse + r);
+      }
+      free(x); free(s); free(mask);
+    }
+  }
+  free(theta); free(cb); free(sb); free(ci); free(si); free(kb); free(ki);
+  return 0;
+}
+
 /* ---- decode (Methodology section 2, on-the-fly correction rotation) ------- */
 
 int jlo_decode_step(jlo_view q_tilde, jlo_view k_cache, jlo_view v_cache, int64_t L, int32_t d,

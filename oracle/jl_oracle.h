@@ -90,6 +90,19 @@ int jlo_bifocal_rows(jlo_view q, jlo_view k, jlo_view v, int64_t L, int32_t d,
                      double* out, double* lse);
 
 /*
+ * Frequency-interpolation variant of the remote window (the pages' ablation:
+ * interpolation, YaRN-style, against position aliasing).  Local pairs
+ * (0 <= i - j < w0) keep base RoPE; every other causal pair scores
+ *     scale * < R'(i) q_i , R'(j) k_j >,   R'(p): angle p * theta_c * lambda_c
+ * with caller-given per-frequency factors lambda [d/2] (lambda_c = 1/G is
+ * position interpolation; a ramp between 1/s and 1 is YaRN's by-parts rule).
+ * No G or f is involved.  Same layout and outputs as jlo_bifocal_rows.
+ */
+int jlo_interp_rows(jlo_view q, jlo_view k, jlo_view v, int64_t L, int32_t d, int32_t n_q_heads,
+                    int32_t n_kv_heads, const int64_t* row_pos, const int32_t* row_head, int64_t n_rows,
+                    int64_t w0, double rope_base, const double* lambda, double scale, double* out, double* lse);
+
+/*
  * The pages' own realisation: three softmax passes merged by inclusion-
  * exclusion on their LogSumExp statistics.
  *   pass 1: local window (0 <= i-j < w0), base positions

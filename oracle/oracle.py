@@ -57,6 +57,8 @@ def lib():
         _lib.jlo_bifocal_rows.argtypes = rows_args + [ctypes.c_int, vp, vp]
         _lib.jlo_bifocal_rows_three_pass.restype = ctypes.c_int
         _lib.jlo_bifocal_rows_three_pass.argtypes = rows_args + [vp, vp, vp]
+        _lib.jlo_interp_rows.restype = ctypes.c_int
+        _lib.jlo_interp_rows.argtypes = [View, View, View, i64, i32, i32, i32, vp, vp, i64, i64, dbl, vp, dbl, vp, vp]
         _lib.jlo_decode_step.restype = ctypes.c_int
         _lib.jlo_decode_step.argtypes = [View, View, View, i64, i32, i32, i32, i64, i64, dbl, dbl,
                                          ctypes.c_int, vp, vp]
@@ -149,6 +151,29 @@ def bifocal_rows(q, k, v, L, row_pos, row_head, *, w0, w_pretrained, rope_base, 
         return out, lse, pl
     rc = lib().jlo_bifocal_rows(qv, kv, vv, L, d, hq, hkv, _ptr(rp), _ptr(rh), n, w0, w_pretrained,
                                 rope_base, sc, int(plain), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments ({rc})")
+    return out, lse
+
+
+def interp_rows(q, k, v, L, row_pos, row_head, *, w0, rope_base, freq_scale, scale=None):
+    """Frequency-interpolation variant: local pairs base RoPE, remote pairs rotated by
+    p * theta_c * freq_scale[c].  Returns (out [n][d], lse [n]) in fp64."""
+    qv, qa = view(q)
+    kv, ka = view(k)
+    vv, va = view(v)
+    d = qa.shape[2]
+    hq, hkv = qa.shape[1], ka.shape[1]
+    rp = np.ascontiguousarray(row_pos, np.int64)
+    rh = np.ascontiguousarray(row_head, np.int32)
+    lam = np.ascontiguousarray(freq_scale, np.float64)
+    assert lam.shape == (d // 2,)
+    n = rp.shape[0]
+    out = np.zeros((n, d), np.float64)
+    lse = np.zeros(n, np.float64)
+    sc = default_scale(d) if scale is None else scale
+    rc = lib().jlo_interp_rows(qv, kv, vv, L, d, hq, hkv, _ptr(rp), _ptr(rh), n, w0, rope_base, _ptr(lam), sc,
+                               _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError(f"oracle rejected arguments ({rc})")
     return out, lse

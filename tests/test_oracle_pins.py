@@ -389,3 +389,43 @@ def test_planted_mistakes_fail_the_pins(kind):
     np.testing.assert_allclose(ob[:, 0], good, atol=1e-12)
     bad = _mutant(kind, q[:, 0], k[:, 0], v[:, 0], L, w0, w_pre, base)
     assert np.abs(bad - ob[:, 0]).max() > 1e-3, kind
+
+
+# ------------------------------------------- frequency-interpolation variant ----
+
+def test_interp_with_unit_factors_is_plain_rope_bit_for_bit():
+    """lambda_c = 1: the remote rotation is the base rotation, so the variant is plain RoPE."""
+    L, d = 60, 16
+    q, k, v = _seq(L, 2, 1, d, 120)
+    pos, head = _all_rows(L, 2)
+    oi, li = O.interp_rows(q, k, v, L, pos, head, w0=7, rope_base=1e4, freq_scale=np.ones(d // 2))
+    op, lp = O.bifocal_rows(q, k, v, L, pos, head, w0=7, w_pretrained=10 ** 6, rope_base=1e4, plain=True)
+    np.testing.assert_array_equal(oi, op)
+    np.testing.assert_array_equal(li, lp)
+
+
+def test_interp_equals_lse_merge_of_library_softmaxes():
+    """Local keys with base RoPE, remote keys with R'(p) (angle p theta_c lambda_c) via complex
+    multiplication; merged on log-sum-exp, by torch SDPA with boolean masks."""
+    L, d, base, w0 = 57, 16, 1e4, 9
+    lam = np.linspace(0.25, 1.0, d // 2)  # a YaRN-like ramp
+    q, k, v = _seq(L, 1, 1, d, 130)
+    pos, head = _all_rows(L, 1)
+    oi, li = O.interp_rows(q, k, v, L, pos, head, w0=w0, rope_base=base, freq_scale=lam)
+    th = base ** (-np.arange(0, d, 2) / d)
+
+    def rot(x, p, scale):
+        z = (x[:, :d // 2] + 1j * x[:, d // 2:]) * np.exp(1j * p[:, None] * (th * scale)[None])
+        return np.concatenate([z.real, z.imag], -1)
+
+    p = np.arange(L).astype(np.float64)
+    dist = np.subtract.outer(np.arange(L), np.arange(L))
+    local, remote = (dist >= 0) & (dist < w0), dist >= w0
+    o1, l1 = _sdpa(rot(q[:, 0], p, 1.0), rot(k[:, 0], p, 1.0), v[:, 0], local)
+    o2, l2 = _sdpa(rot(q[:, 0], p, lam), rot(k[:, 0], p, lam), v[:, 0], remote)
+    has2 = remote.any(1)
+    lse = np.where(has2, np.logaddexp(l1, np.where(has2, l2, -np.inf)), l1)
+    ref = np.exp(l1 - lse)[:, None] * o1 + np.where(has2, np.exp(np.where(has2, l2, 0) - lse), 0)[:, None] * \
+        np.where(has2[:, None], o2, 0)
+    np.testing.assert_allclose(oi, ref, atol=1e-12)
+    np.testing.assert_allclose(li, lse, atol=1e-12)
