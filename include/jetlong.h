@@ -89,6 +89,30 @@ jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t 
                          jl_stream_t stream);
 
 /*
+ * Scaled RoPE tables for the frequency-interpolation variant:
+ * cos/sin(p * theta_c * freq_scale[c]), fp64 angle rounded to fp32 once.
+ * freq_scale: HOST array of head_dim/2 positive factors (1/G for position
+ * interpolation; a ramp between 1/s and 1 for a YaRN-style by-parts rule).
+ */
+jl_status jl_rope_tables_scaled(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
+                                const double* freq_scale, jl_stream_t stream);
+
+/*
+ * Frequency-interpolation variant of the remote window (the pages' ablation of
+ * position aliasing against interpolation, Results; kernel only).  Local pairs
+ * (0 <= i-j < w0) keep base RoPE from cos_tab/sin_tab; every other causal pair
+ * scores <R'(i) q, R'(j) k> with R' read from cos_rem/sin_rem at the raw
+ * positions (from jl_rope_tables_scaled).  No G or f: the caller's table sets
+ * the compression.  Same layout, conventions and kernel as jl_bifocal_prefill;
+ * n_rem_rows >= max_seqlen.
+ */
+jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                            int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                            int32_t w0, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                            const float* cos_rem, const float* sin_rem, int64_t n_rem_rows, float softmax_scale,
+                            void* out, float* lse, jl_stream_t stream);
+
+/*
  * Bifocal prefill (Methodology section 2, inclusion-exclusion attention merge).
  * Computes, for every token i of every packed sequence and every query head,
  *   out = softmax_j(scale * s(i, j)) V   over j <= i, with s the routed score,

@@ -434,6 +434,49 @@ jl_status jl_selftest_wait_timeout(int64_t limit_cycles, jl_stream_t stream) {
   return ok();
 }
 
+jl_status jl_rope_tables_scaled(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
+                                const double* freq_scale, jl_stream_t stream) {
+  if (!cos_out || !sin_out || !freq_scale) return fail(JL_ERR_INVALID, "null pointer argument");
+  if (n_pos < 1) return fail(JL_ERR_INVALID, "n_pos must be >= 1 (got %lld)", (long long)n_pos);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(JL_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (!(rope_base > 1.0)) return fail(JL_ERR_INVALID, "rope_base must be > 1");
+  if (!aligned16(cos_out) || !aligned16(sin_out)) return fail(JL_ERR_INVALID, "tables must be 16-byte aligned");
+  jl::FreqScale fs{};
+  for (int c = 0; c < head_dim / 2; ++c) {
+    if (!(freq_scale[c] > 0.0)) return fail(JL_ERR_INVALID, "freq_scale[%d] must be > 0", c);
+    fs.lambda[c] = freq_scale[c];
+  }
+  const int half = head_dim / 2;
+  const int64_t blocks64 = (n_pos * half + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(blocks64 < 148 * 64 ? blocks64 : 148 * 64);
+  jl::jl_rope_table_scaled_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(cos_out, sin_out, n_pos,
+                                                                                              half, rope_base, fs);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "scaled table launch");
+  return ok();
+}
+
+jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                            int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                            int32_t w0, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                            const float* cos_rem, const float* sin_rem, int64_t n_rem_rows, float softmax_scale,
+                            void* out, float* lse, jl_stream_t stream) {
+  if (!cos_rem || !sin_rem) return fail(JL_ERR_INVALID, "null remote table");
+  if (n_rem_rows < max_seqlen)
+    return fail(JL_ERR_INVALID, "n_rem_rows (%lld) must be >= max_seqlen (%d)", (long long)n_rem_rows, max_seqlen);
+  if (!aligned16(cos_rem) || !aligned16(sin_rem)) return fail(JL_ERR_INVALID, "tables must be 16-byte aligned");
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0, 1, 0,
+                               cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm, &empty);
+  if (s != JL_OK || empty) return s;
+  prm.cos_rem = cos_rem;
+  prm.sin_rem = sin_rem;
+  prm.n_rem_rows = n_rem_rows;
+  return launch_prefill_any(q, k, v, prm, head_dim, reinterpret_cast<cudaStream_t>(stream));
+}
+
 jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,
                          jl_stream_t stream) {
   if (!cos_out || !sin_out) return fail(JL_ERR_INVALID, "null table pointer");

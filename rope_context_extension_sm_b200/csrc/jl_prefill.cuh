@@ -63,6 +63,9 @@ struct PrefillParams {
   int32_t plain;
   int32_t mode;          // 0: fused bifocal / plain; 1: pass 1 alone; 3: pass 3 alone (see TileSchedule)
   int32_t cached;        // keys/values come from a base-RoPE cache (chunked prefill)
+  const float* cos_rem;  // frequency-interpolation variant: remote pairs rotate by these
+  const float* sin_rem;  // rows at their raw positions (cos/sin(p theta_c lambda_c)); NULL = aliasing
+  int64_t n_rem_rows;
   const int32_t* past_lens;  // cached: tokens in each cache entry before this chunk
   int64_t cache_stride;      // cached: positions per cache entry
   float scale_log2;      // softmax scale * log2(e)
@@ -149,17 +152,21 @@ struct RotFactor {
   float c[NF], s[NF];
 };
 
+// Factor of table row `row` (base table, or the interpolated remote table when rem).
 template <int D>
-__device__ __forceinline__ void load_factor(RotFactor<D>& f, const PrefillParams& p, int64_t row, int lane) {
-  const int64_t max_row = p.n_tab_rows - 1;
+__device__ __forceinline__ void load_factor(RotFactor<D>& f, const PrefillParams& p, int64_t row, int lane,
+                                            bool rem = false) {
+  const float* ct = rem ? p.cos_rem : p.cos_tab;
+  const float* st = rem ? p.sin_rem : p.sin_tab;
+  const int64_t max_row = (rem ? p.n_rem_rows : p.n_tab_rows) - 1;
   row = row > max_row ? max_row : row;  // only rows past every sequence end are clamped
   if constexpr (D == 128) {
-    const float2 cc = __ldg(reinterpret_cast<const float2*>(p.cos_tab + row * 64 + 2 * lane));
-    const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + row * 64 + 2 * lane));
+    const float2 cc = __ldg(reinterpret_cast<const float2*>(ct + row * 64 + 2 * lane));
+    const float2 ss = __ldg(reinterpret_cast<const float2*>(st + row * 64 + 2 * lane));
     f.c[0] = cc.x; f.c[1] = cc.y; f.s[0] = ss.x; f.s[1] = ss.y;
   } else {
-    f.c[0] = __ldg(p.cos_tab + row * 32 + lane);
-    f.s[0] = __ldg(p.sin_tab + row * 32 + lane);
+    f.c[0] = __ldg(ct + row * 32 + lane);
+    f.s[0] = __ldg(st + row * 32 + lane);
   }
 }
 
@@ -349,11 +356,12 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   const int L = past + n_rows;                      // sequence length after this chunk
   const int q_tok0 = seq0 + qt * kBM;               // packed index of the block's first query
 
+  const bool interp = p.cos_rem != nullptr;  // remote pairs: interpolated table, no aliasing
   int G = 1;
-  if (!p.plain) G = max(1, (L + p.w_pre - 1) / p.w_pre);
+  if (!p.plain && !interp) G = max(1, (L + p.w_pre - 1) / p.w_pre);
   // G = 1 (or plain): remote scores equal base scores, every pair runs as local.
   // The literal passes keep the real window.
-  const int w0_eff = (p.mode == 0 && (p.plain || G == 1)) ? (1 << 30) : p.w0;
+  const int w0_eff = (p.mode == 0 && !interp && (p.plain || G == 1)) ? (1 << 30) : p.w0;
   TileSchedule sc;
   sc.init(past + qt * kBM, L, w0_eff, p.mode == 0);
   // Pass 3 rotates its (local-window) visits by the remote positions.
@@ -530,8 +538,9 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   } else if (Lay::rot_index(warp) >= 0) {
     // ------------------------------------------------------------ rotation
     const int rw = Lay::rot_index(warp);
-    RotFactor<D> step;  // e^{i theta_c}: table row 1
+    RotFactor<D> step, step_rem;  // e^{i theta_c} (row 1 of the base table) and of the interpolated table
     load_factor<D>(step, p, 1, lane);
+    if (interp) load_factor<D>(step_rem, p, 1, lane, true);
     auto key_anchor = [&](int n) -> int64_t {
       if (p.cached) {  // correction index n_j = j - f(j) of the slice's first cached key
         const int j = sc.kt(n) * kBN + 32 * rw;
@@ -540,25 +549,28 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       return slice_anchor_row(sc.kt(n) * kBN, rw, (sc.remote(n) || local_uses_remote) ? G : 1);
     };
     RotFactor<D> fk_next;
-    load_factor<D>(fk_next, p, key_anchor(0), lane);
+    load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
-      const int g = (remote || local_uses_remote) ? G : 1;
+      const bool rem_tab = interp && remote;  // interpolated rows at raw positions
+      const int g = (!interp && (remote || local_uses_remote)) ? G : 1;
+      const RotFactor<D>& stp = rem_tab ? step_rem : step;
       if (sc.phase_start(n)) {
         RotFactor<D> fq;
-        load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane);
+        load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane, rem_tab);
         if (!mbar_wait(&bars->q_full, n == 0 ? 0 : 1, abort)) break;
-        for (int t = 0; t < NQT; ++t) rotate_slice_any<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, step, lane);
+        for (int t = 0; t < NQT; ++t) rotate_slice_any<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, stp, lane);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_ready);
       }
       const RotFactor<D> fk = fk_next;
-      if (n + 1 < sc.n_virt) load_factor<D>(fk_next, p, key_anchor(n + 1), lane);  // prefetch a tile ahead
+      if (n + 1 < sc.n_virt)  // prefetch a tile ahead
+        load_factor<D>(fk_next, p, key_anchor(n + 1), lane, interp && sc.remote(n + 1));
       const int s = n % kStages;
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
       if (!p.cached) {
-        rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane);
+        rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, stp, lane);
       } else if (g > 1) {  // cached keys are base-rotated: local visits use them as they are
         switch (g) {
           case 2: correct_slice<D, 2>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane); break;

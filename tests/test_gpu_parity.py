@@ -551,3 +551,42 @@ def test_paged_cache_writers_match_contiguous(jl):
         jl.jl_sync_status()
     assert err.value.status == jl.JL_ERR_INVALID
     jl.jl_sync_status()
+
+
+# ------------------------------------------- frequency-interpolation variant ----
+
+def _yarn_ramp(d, s, base, w_pre, alpha=1.0, beta=32.0):
+    """A YaRN-style by-parts factor per frequency: 1/s for long wavelengths, 1 for short."""
+    th = base ** (-np.arange(0, d, 2) / d)
+    r = w_pre * th / (2 * np.pi)  # rotations within the pretraining window
+    gamma = np.clip((r - alpha) / (beta - alpha), 0.0, 1.0)
+    return (1 - gamma) / s + gamma
+
+
+INTERP = [
+    ("pi_G4", (1000,), 8, 2, 128, 100, "pi", 4.0),
+    ("yarn_s4", (1000,), 8, 2, 128, 100, "yarn", 4.0),
+    ("yarn_varlen", (300, 129, 700), 4, 2, 128, 64, "yarn", 3.0),
+    ("pi_d64_w0_0", (400,), 3, 1, 64, 0, "pi", 2.0),
+]
+
+
+@pytest.mark.parametrize("case", INTERP, ids=[c[0] for c in INTERP])
+def test_interp_prefill_matches_oracle(jl, case):
+    name, seqlens, hq, hkv, d, w0, kind, s = case
+    cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, 256, 1e4, True)
+    lam = np.full(d // 2, 1.0 / s) if kind == "pi" else _yarn_ramp(d, s, cfg.rope_base, 256)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    n = max(cfg.max_seqlen, 1)
+    cos, sin = _tables(jl, n, d, cfg.rope_base)
+    cr, sr = jl.jl_rope_tables_scaled(n, d, cfg.rope_base, lam)
+    out, lse = jl.jl_interp_prefill(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), cfg.max_seqlen, w0, cos, sin, cr, sr)
+    jl.jl_sync_status()
+    out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    for b, L in enumerate(seqlens):
+        s0 = int(cu[b])
+        pos = np.repeat(np.arange(L), hq)
+        head = np.tile(np.arange(hq), L)
+        ro, rl = O.interp_rows(I.bf16_bits(q[s0:s0 + L]), I.bf16_bits(k[s0:s0 + L]), I.bf16_bits(v[s0:s0 + L]), L,
+                               pos, head, w0=w0, rope_base=cfg.rope_base, freq_scale=lam)
+        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{name} seq {b}")
