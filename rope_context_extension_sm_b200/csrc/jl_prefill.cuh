@@ -194,12 +194,14 @@ __device__ __forceinline__ void rotate_row(uint8_t* tile, int r, const RotFactor
     __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
     const float2 a = __bfloat1622float2(*plo);
     const float2 b = __bfloat1622float2(*phi);
-    const float s0 = sg * f.s[0], s1 = sg * f.s[1];
+    // ya = a c - b s, yb = b c + a s on packed pairs (two frequencies per instruction)
+    const uint64_t c2 = f2_pack(f.c[0], f.c[1]);
+    const uint64_t s2 = f2_pack(sg * f.s[0], sg * f.s[1]);
+    const uint64_t ns2 = f2_pack(-sg * f.s[0], -sg * f.s[1]);
+    const uint64_t a2 = f2_pack(a.x, a.y), b2 = f2_pack(b.x, b.y);
     float2 ya, yb;
-    ya.x = a.x * f.c[0] - b.x * s0;
-    yb.x = b.x * f.c[0] + a.x * s0;
-    ya.y = a.y * f.c[1] - b.y * s1;
-    yb.y = b.y * f.c[1] + a.y * s1;
+    f2_unpack(f2_fma(b2, ns2, f2_mul(a2, c2)), ya.x, ya.y);
+    f2_unpack(f2_fma(a2, s2, f2_mul(b2, c2)), yb.x, yb.y);
     *plo = __float22bfloat162_rn(ya);
     *phi = __float22bfloat162_rn(yb);
   } else {
@@ -312,19 +314,25 @@ __device__ __forceinline__ void correct_slice(uint8_t* tile, int rw, int kbase, 
 template <bool MASK>
 __device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[64], uint32_t (&pk)[32], int col0, float sl2,
                                               float neg_m, int keep_lo, int keep_hi, float& lsum, float& lsum2) {
+  const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+  uint64_t acc = f2_pack(lsum, lsum2);
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m));
-    float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m));
+    // (s0, s1) * scale - m in one packed FMA, two ex2, one packed add into the row sums
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), scale2, negm2);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    float p0 = ex2_approx(x0);
+    float p1 = ex2_approx(x1);
     if constexpr (MASK) {
       const int col = col0 + 2 * e;
       p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
       p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
     }
-    lsum += p0;
-    lsum2 += p1;
+    acc = f2_add(acc, f2_pack(p0, p1));
     pk[e] = pack_bf16x2(p0, p1);
   }
+  f2_unpack(acc, lsum, lsum2);
 }
 
 template <int D, int NQT>
