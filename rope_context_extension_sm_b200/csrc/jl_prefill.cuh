@@ -471,78 +471,89 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      auto issue_s = [&](int t, int s) {
-        const uint32_t qa = q_addr + t * Lay::kTileBytes;
-        const uint32_t ka = k_addr + s * Lay::kTileBytes;
+    // The whole warp runs the loop, so every operand stays warp-uniform; one
+    // elected lane issues each tcgen05 instruction.  Descriptors are formed
+    // once: the descriptor of (base + off) is that of base plus off / 16 (the
+    // start-address field, which cannot carry below 256 KB of shared memory).
+    const bool leader = elect_one();
+    const uint64_t dq0 = sdesc_kmajor_sw128(smem_u32(sQ));
+    const uint64_t dk0 = sdesc_kmajor_sw128(smem_u32(sK));
+    const uint64_t dv0 = sdesc_mnmajor_sw128(smem_u32(sV), 16384);
+    auto issue_s = [&](int t, int s) {
+      const uint64_t qd = dq0 + static_cast<uint32_t>((t * Lay::kTileBytes) >> 4);
+      const uint64_t kd = dk0 + static_cast<uint32_t>((s * Lay::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::kBoxBytes + (kk & 3) * 32;
-          umma_ss(tmem + t * 128, sdesc_kmajor_sw128(qa + off), sdesc_kmajor_sw128(ka + off), kIdescS, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t va = v_addr + s * Lay::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < PSTEPS; ++kk)
-          umma_ts(tmem + NQT * 128 + t * D, tmem + t * 128 + kk * 8, sdesc_mnmajor_sw128(va + kk * 2048, 16384),
-                  kIdescO, (acc || kk > 0) ? 1u : 0u);
-      };
-      int n = 0;
-      bool ok = true;
-      for (; n < sc.n_virt && ok; ++n) {
-        if (sc.phase_start(n)) {
-          if (!(ok = mbar_wait(&bars->q_ready, n == 0 ? 0 : 1, abort))) break;
-          tc_fence_after();
-        }
-        const int s = n % kStages;
-        const uint32_t u = n / kStages;
-        if (!(ok = mbar_wait(&bars->k_ready[s], u & 1, abort))) break;
-        tc_fence_after();
-        issue_s(0, s);
-        umma_commit(&bars->s_full[0]);
-        if (NQT == 2) {
-          if (n > 0) {
-            const int sp = (n - 1) % kStages;
-            if (!(ok = mbar_wait(&bars->p_ready[1], (n - 1) & 1, abort))) break;
-            tc_fence_after();
-            if (!(ok = mbar_wait(&bars->v_full[sp], ((n - 1) / kStages) & 1, abort))) break;
-            issue_pv(1, sp, n - 1 > 0);
-            umma_commit(&bars->v_empty[sp]);
-          }
-          issue_s(1, s);
-          umma_commit(&bars->s_full[1]);
-        }
-        umma_commit(&bars->k_empty[s]);
-        if (sc.phase_end(n)) umma_commit(&bars->q_empty);
-        if (!(ok = mbar_wait(&bars->p_ready[0], n & 1, abort))) break;
-        tc_fence_after();
-        if (!(ok = mbar_wait(&bars->v_full[s], u & 1, abort))) break;
-        issue_pv(0, s, n > 0);
-        if (NQT == 1) umma_commit(&bars->v_empty[s]);
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        constexpr uint32_t kBox16 = Lay::kBoxBytes >> 4;
+        const uint32_t off = (kk >> 2) * kBox16 + (kk & 3) * 2;
+        if (leader) umma_ss(tmem + t * 128, qd + off, kd + off, kIdescS, kk > 0);
       }
-      if (ok && NQT == 2) {
-        const int nl = sc.n_virt - 1;
-        const int sl = nl % kStages;
-        ok = mbar_wait(&bars->p_ready[1], nl & 1, abort);
-        if (ok) {
+    };
+    auto issue_pv = [&](int t, int s, bool acc) {
+      const uint64_t vd = dv0 + static_cast<uint32_t>((s * Lay::kTileBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < PSTEPS; ++kk)
+        if (leader)
+          umma_ts(tmem + NQT * 128 + t * D, tmem + t * 128 + kk * 8, vd + kk * (2048 >> 4), kIdescO,
+                  (acc || kk > 0) ? 1u : 0u);
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) umma_commit(bar);
+    };
+    int n = 0;
+    bool ok = true;
+    for (; n < sc.n_virt && ok; ++n) {
+      if (sc.phase_start(n)) {
+        if (!(ok = warp_wait(&bars->q_ready, n == 0 ? 0 : 1, abort))) break;
+        tc_fence_after();
+      }
+      const int s = n % kStages;
+      const uint32_t u = n / kStages;
+      if (!(ok = warp_wait(&bars->k_ready[s], u & 1, abort))) break;
+      tc_fence_after();
+      issue_s(0, s);
+      commit(&bars->s_full[0]);
+      if (NQT == 2) {
+        if (n > 0) {
+          const int sp = (n - 1) % kStages;
+          if (!(ok = warp_wait(&bars->p_ready[1], (n - 1) & 1, abort))) break;
           tc_fence_after();
-          ok = mbar_wait(&bars->v_full[sl], (nl / kStages) & 1, abort);
+          if (!(ok = warp_wait(&bars->v_full[sp], ((n - 1) / kStages) & 1, abort))) break;
+          issue_pv(1, sp, n - 1 > 0);
+          commit(&bars->v_empty[sp]);
         }
-        if (ok) {
-          issue_pv(1, sl, nl > 0);
-          umma_commit(&bars->v_empty[sl]);
-        }
+        issue_s(1, s);
+        commit(&bars->s_full[1]);
+      }
+      commit(&bars->k_empty[s]);
+      if (sc.phase_end(n)) commit(&bars->q_empty);
+      if (!(ok = warp_wait(&bars->p_ready[0], n & 1, abort))) break;
+      tc_fence_after();
+      if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
+      issue_pv(0, s, n > 0);
+      if (NQT == 1) commit(&bars->v_empty[s]);
+    }
+    if (ok && NQT == 2) {
+      const int nl = sc.n_virt - 1;
+      const int sl = nl % kStages;
+      ok = warp_wait(&bars->p_ready[1], nl & 1, abort);
+      if (ok) {
+        tc_fence_after();
+        ok = warp_wait(&bars->v_full[sl], (nl / kStages) & 1, abort);
       }
       if (ok) {
-        umma_commit(&bars->o_final[0]);
-        if (NQT == 2) umma_commit(&bars->o_final[1]);
+        issue_pv(1, sl, nl > 0);
+        commit(&bars->v_empty[sl]);
       }
-      // Every issued MMA must finish before TMEM is released.
-      umma_commit(&bars->teardown);
-      mbar_wait_bounded(&bars->teardown, 0);
     }
+    if (ok) {
+      commit(&bars->o_final[0]);
+      if (NQT == 2) commit(&bars->o_final[1]);
+    }
+    // Every issued MMA must finish before TMEM is released.
+    commit(&bars->teardown);
+    mbar_wait_bounded(&bars->teardown, 0);
+    __syncwarp();
   } else if (Lay::rot_index(warp) >= 0) {
     // ------------------------------------------------------------ rotation
     const int rw = Lay::rot_index(warp);
