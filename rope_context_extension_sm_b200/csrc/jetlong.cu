@@ -91,10 +91,20 @@ jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::
   auto kern = jl::jl_prefill_kernel<D, NQT>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
+  static int launch_regs = 0;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+    cudaFuncAttributes fa{};
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, kern);
+    launch_regs = fa.numRegs;
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
+  // The kernel moves registers between its warpgroups (setmaxnreg); the softmax
+  // warpgroups' increase would wait forever if the launch allocation could not
+  // cover the split, so such a build is refused here rather than launched.
+  if (Lay::kSplitRegs && static_cast<int64_t>(launch_regs) * Lay::kThreads < Lay::kRegsNeeded)
+    return fail(JL_ERR_UNSUPPORTED, "prefill kernel built with %d registers per thread; the register split needs %u",
+                launch_regs, Lay::kRegsLaunch);
   const int64_t blocks = static_cast<int64_t>(prm.n_qtiles) * prm.batch * prm.Hkv * prm.slots;
   if (blocks > 0x7fffffff) return fail(JL_ERR_UNSUPPORTED, "prefill grid too large (%lld blocks)", (long long)blocks);
   kern<<<static_cast<unsigned>(blocks), Lay::kThreads, Lay::kAlloc, st>>>(tq, tk, tv, prm);

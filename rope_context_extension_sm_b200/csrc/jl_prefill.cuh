@@ -84,10 +84,24 @@ struct PrefillLayout {
   static constexpr int kColsUsed = NQT * 128 + NQT * D;
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
   static constexpr int kRotWarps = 4;
-  static constexpr int kThreads = 32 * (2 + kRotWarps) + NQT * 128;
-  // warps: 0 producer, 1 MMA, 2-3 rotation, 4 .. 4+4NQT-1 softmax, then 2 more rotation warps
+  // warps: 0 producer, 1 MMA, 2-3 rotation, 4 .. kR0-1 softmax (one warpgroup
+  // per query head), kR0 and kR0+1 rotation, kR0+2 and kR0+3 idle (every
+  // warpgroup is complete, as the register split requires).
+  static constexpr int kR0 = 4 + 4 * NQT;
+  static constexpr int kWarps = kR0 + 4;
+  static constexpr int kThreads = 32 * kWarps;
+  // The softmax warpgroups hold a whole 128-column score row in registers.  The
+  // block is launched at kRegsLaunch registers per thread; the producer / MMA /
+  // rotation warpgroups give theirs down to kRegsOther and the softmax
+  // warpgroups take kRegsSoftmax.  Two heads: 128 x (2 x 200 + 2 x 56) = 512 x 128.
+  static constexpr bool kSplitRegs = true;
+  static constexpr uint32_t kRegsLaunch = (65536 / kThreads) & ~7u;
+  static constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 56;
+  static constexpr uint32_t kRegsNeeded = 128 * (NQT * kRegsSoftmax + (kWarps / 4 - NQT) * kRegsOther);
+  static_assert(kRegsNeeded <= kThreads * kRegsLaunch, "register split exceeds the launch allocation");
+  __device__ static bool softmax_warp(int warp) { return warp >= 4 && warp < kR0; }
   __device__ static int rot_index(int warp) {
-    return warp < 4 ? warp - 2 : (warp >= 4 + 4 * NQT ? warp - (4 + 4 * NQT) + 2 : -1);
+    return (warp == 2 || warp == 3) ? warp - 2 : ((warp == kR0 || warp == kR0 + 1) ? warp - kR0 + 2 : -1);
   }
 };
 
@@ -308,16 +322,16 @@ __device__ __forceinline__ void correct_slice(uint8_t* tile, int rw, int kbase, 
   }
 }
 
-// Softmax pass B on one 64-column chunk: p = 2^(s * sl2 - m) (zero outside
-// [keep_lo + 1, keep_hi] when MASK), packed to bf16 pairs; returns the two
-// partial row sums.  Straight-line code: no branch inside the chunk.
-template <bool MASK>
-__device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[64], uint32_t (&pk)[32], int col0, float sl2,
+// p = 2^(s * sl2 - m) over NC score columns (zero outside [keep_lo + 1,
+// keep_hi] when MASK), packed to bf16 pairs; accumulates the two partial row
+// sums.  Straight-line code: no branch inside.
+template <bool MASK, int NC>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[NC], uint32_t (&pk)[NC / 2], int col0, float sl2,
                                               float neg_m, int keep_lo, int keep_hi, float& lsum, float& lsum2) {
   const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
   uint64_t acc = f2_pack(lsum, lsum2);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
+  for (int e = 0; e < NC / 2; ++e) {
     // (s0, s1) * scale - m in one packed FMA, two ex2, one packed add into the row sums
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), scale2, negm2);
     float x0, x1;
@@ -429,8 +443,14 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // Register split: each role's first instruction, executed by the whole warp
+  // (every warp of a warpgroup takes the same share).
+  auto give_regs = [] {
+    if constexpr (Lay::kSplitRegs) setmaxnreg_dec<Lay::kRegsOther>();
+  };
 
   if (warp == 0) {
+    give_regs();
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -470,6 +490,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         }
     }
   } else if (warp == 1) {
+    give_regs();
     // ---------------------------------------------------------- MMA issuer
     // The whole warp runs the loop, so every operand stays warp-uniform; one
     // elected lane issues each tcgen05 instruction.  Descriptors are formed
@@ -555,6 +576,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     mbar_wait_bounded(&bars->teardown, 0);
     __syncwarp();
   } else if (Lay::rot_index(warp) >= 0) {
+    give_regs();
     // ------------------------------------------------------------ rotation
     const int rw = Lay::rot_index(warp);
     RotFactor<D> step, step_rem;  // e^{i theta_c} (row 1 of the base table) and of the interpolated table
@@ -601,7 +623,8 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);
     }
-  } else {
+  } else if (Lay::softmax_warp(warp)) {
+    if constexpr (Lay::kSplitRegs) setmaxnreg_inc<Lay::kRegsSoftmax>();
     // ------------------------------------------------------ softmax + epilogue
     const int t = (warp - 4) >> 2;  // query head slot
     const int wq = warp & 3;        // TMEM lane quarter
@@ -617,7 +640,9 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     for (int n = 0; n < sc.n_virt; ++n) {
       if (!(ok = mbar_wait(&bars->s_full[t], n & 1, abort))) break;
       tc_fence_after();
-      // Pass A: row max over the (masked) scores, 64 columns at a time.
+      // The whole score row in registers: one TMEM round trip per tile.
+      uint32_t sr[128];
+      tmem_ld128(t_s, sr);
       const bool msk = sc.masked(n);
       const int hi = i - sc.kt(n) * kBN;  // causal: keep column c <= hi
       const int edge = hi - sc.w0;        // remote keeps c <= edge, local keeps c > edge
@@ -625,25 +650,19 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const int keep_lo = msk ? (rem ? -1 : edge) : -1;     // keep c > keep_lo
       const int keep_hi = msk ? (rem ? edge : hi) : kBN;    // keep c <= keep_hi
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sr[64];
-        tmem_ld64(t_s + c * 64, sr);
-        if (msk) {
+      if (msk) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int col = c * 64 + e;
-            mx = (col > keep_lo && col <= keep_hi) ? fmaxf(mx, __uint_as_float(sr[e])) : mx;
-          }
-        } else {
-          float m2 = -INFINITY;
+        for (int e = 0; e < 128; ++e) mx = (e > keep_lo && e <= keep_hi) ? fmaxf(mx, __uint_as_float(sr[e])) : mx;
+      } else {
+        float m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 64; e += 4) {
-            mx = fmax3(mx, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
-            m2 = fmax3(m2, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
-          }
-          mx = fmaxf(mx, m2);
+        for (int e = 0; e < 128; e += 8) {
+          mx = fmax3(mx, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+          m1 = fmax3(m1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+          m2 = fmax3(m2, __uint_as_float(sr[e + 4]), __uint_as_float(sr[e + 5]));
+          m3 = fmax3(m3, __uint_as_float(sr[e + 6]), __uint_as_float(sr[e + 7]));
         }
+        mx = fmaxf(fmaxf(mx, m1), fmaxf(m2, m3));
       }
       const float m_new = fmaxf(m_run, mx * sl2);
       // Lazy rescale: keep the stale max unless the new one exceeds it by > 8 (x256).
@@ -651,28 +670,12 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const float alpha = resc ? ex2_approx(m_run - m_new) : 1.f;
       if (resc || m_run == -INFINITY) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // Pass B: P = 2^(s * scale_log2 - m), written back over S as bf16 pairs.
-      // Chunk c reads S columns [64c, 64c+64) and writes P columns [32c, 32c+32);
-      // every write lands on S columns that were already read.
+      // P = 2^(s * scale_log2 - m) as bf16 pairs over S columns [0, 64).
       float lsum = 0.f, lsum2 = 0.f;
-      const float neg_m = -m_use;
-      if (msk) {
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sr[64], pk[32];
-          tmem_ld64(t_s + c * 64, sr);
-          softmax_chunk<true>(sr, pk, c * 64, sl2, neg_m, keep_lo, keep_hi, lsum, lsum2);
-          tmem_st32(t_s + c * 32, pk);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sr[64], pk[32];
-          tmem_ld64(t_s + c * 64, sr);
-          softmax_chunk<false>(sr, pk, c * 64, sl2, neg_m, keep_lo, keep_hi, lsum, lsum2);
-          tmem_st32(t_s + c * 32, pk);
-        }
-      }
+      uint32_t pk[64];
+      if (msk) softmax_chunk<true, 128>(sr, pk, 0, sl2, -m_use, keep_lo, keep_hi, lsum, lsum2);
+      else softmax_chunk<false, 128>(sr, pk, 0, sl2, -m_use, keep_lo, keep_hi, lsum, lsum2);
+      tmem_st64(t_s, pk);
       lsum += lsum2;
       l_run = l_run * alpha + lsum;
       // O_t *= alpha for the rows whose max moved (PV_t(n-1) is complete: it was
@@ -726,6 +729,8 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       }
     }
   }
+
+  if (warp >= Lay::kR0 + 2) give_regs();  // idle warps (two-head layout) still give their share
 
   // ---- teardown: every role is done; TMEM is released by its allocator warp ----
   tc_fence_before();
