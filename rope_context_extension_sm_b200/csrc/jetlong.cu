@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -194,27 +195,27 @@ size_t three_pass_ws_bytes(int64_t total_tokens, int32_t Hq, int32_t head_dim) {
 // ------------------------------------------------------------------ decode --
 
 // Tensor-core decode (head_dim 128, up to 16 query heads per KV head) splits the
-// keys in chunks of whole 128-key tiles, sized for about four waves of CTAs; the
-// other shapes use the CUDA-core split kernel.
+// keys in chunks of whole 128-key tiles, sized for one wave of CTAs; the other
+// shapes use the CUDA-core split kernel.
 bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) { return head_dim == 128 && Hq / Hkv <= 16; }
 
 // Keys per split.  CUDA-core kernel: a power of two in [64, 512].  Tensor-core
-// kernel: whole 128-key tiles, sized so that 8 KV heads x B entries fill the 148
-// SMs of a B200 in one wave (one CTA per SM; a single wave keeps each CTA's
-// K/V pipeline full instead of paying a cold start per short chunk).  The split
-// count depends only on B and max_seqlen, never on the head counts, so the
-// workspace-size query below can bound it.
+// kernel: whole 128-key tiles, as many splits per (entry, KV head) as fit the
+// 148 SMs of a B200 in ONE wave (one CTA per SM): a CTA left over for a second
+// wave would run after all the others and set the kernel's time.
+constexpr int64_t kSMs = 148;
+
 int chunk_cuda_core(int32_t max_seqlen) {
   int c = 64;
   while (c < 512 && static_cast<int64_t>(c) * 256 < max_seqlen) c *= 2;
   return c;
 }
 
-int chunk_tc(int32_t B, int32_t max_seqlen) {
+int chunk_tc(int32_t B, int32_t Hkv, int32_t max_seqlen) {
   const int64_t tiles = (static_cast<int64_t>(max_seqlen) + jl::kDecTile - 1) / jl::kDecTile;
-  const int64_t want_ctas = 148;
-  int64_t per = (tiles * 8 * B + want_ctas - 1) / want_ctas;
-  per = per < 1 ? 1 : per;
+  const int64_t ctas_per_split = static_cast<int64_t>(Hkv) * B;
+  const int64_t n_target = std::max<int64_t>(1, kSMs / std::max<int64_t>(1, ctas_per_split));
+  const int64_t per = std::max<int64_t>(1, (tiles + n_target - 1) / n_target);
   return static_cast<int>(per * jl::kDecTile);
 }
 
@@ -282,12 +283,14 @@ size_t ws_bytes_for(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen,
   return static_cast<size_t>(B) * n_split * Hq * (head_dim + 2) * sizeof(float);
 }
 
-// Upper bound over both decode kernels (the query does not know Hkv, which picks the kernel).
+// Upper bound over both decode kernels and every KV-head count the query heads
+// allow (the query does not know Hkv, which picks the kernel and the split).
 size_t decode_ws_bytes(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen) {
   if (B <= 0 || Hq <= 0 || head_dim <= 0 || max_seqlen <= 0) return 0;
   size_t n = ws_bytes_for(B, Hq, head_dim, max_seqlen, chunk_cuda_core(max_seqlen));
-  if (head_dim == 128) {
-    const size_t t = ws_bytes_for(B, Hq, head_dim, max_seqlen, chunk_tc(B, max_seqlen));
+  for (int32_t hkv = 1; hkv <= Hq; ++hkv) {
+    if (Hq % hkv != 0 || !decode_uses_tc(head_dim, Hq, hkv)) continue;
+    const size_t t = ws_bytes_for(B, Hq, head_dim, max_seqlen, chunk_tc(B, hkv, max_seqlen));
     n = t > n ? t : n;
   }
   return n;
@@ -344,7 +347,7 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
   prm.w0 = w0;
   prm.w_pre = w_pretrained;
   prm.plain = plain;
-  prm.chunk = decode_uses_tc(head_dim, Hq, Hkv) ? chunk_tc(B, max_seqlen) : chunk_cuda_core(max_seqlen);
+  prm.chunk = decode_uses_tc(head_dim, Hq, Hkv) ? chunk_tc(B, Hkv, max_seqlen) : chunk_cuda_core(max_seqlen);
   prm.n_split = (max_seqlen + prm.chunk - 1) / prm.chunk;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   prm.scale_log2 = scale * 1.4426950408889634f;

@@ -77,11 +77,12 @@ __device__ __forceinline__ void rotate_row_neg(uint8_t* tile, int r, const float
   __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
   const float2 a = __bfloat1622float2(*plo);
   const float2 b = __bfloat1622float2(*phi);
+  // ya = a c + b s, yb = b c - a s on packed pairs (two frequencies per instruction)
+  const uint64_t c2 = f2_pack(c[0], c[1]), s2 = f2_pack(s[0], s[1]);
+  const uint64_t a2 = f2_pack(a.x, a.y), b2 = f2_pack(b.x, b.y);
   float2 ya, yb;
-  ya.x = a.x * c[0] + b.x * s[0];
-  yb.x = b.x * c[0] - a.x * s[0];
-  ya.y = a.y * c[1] + b.y * s[1];
-  yb.y = b.y * c[1] - a.y * s[1];
+  f2_unpack(f2_fma(b2, s2, f2_mul(a2, c2)), ya.x, ya.y);
+  f2_unpack(f2_sub(f2_mul(b2, c2), f2_mul(a2, s2)), yb.x, yb.y);
   *plo = __float22bfloat162_rn(ya);
   *phi = __float22bfloat162_rn(yb);
 }
@@ -89,12 +90,15 @@ __device__ __forceinline__ void rotate_row_neg(uint8_t* tile, int r, const float
 // (c, s) <- (c, s) * e^{i theta} when adv, else unchanged (select, no branch).
 __device__ __forceinline__ void step_factor(float (&c)[2], float (&s)[2], const float (&st_c)[2],
                                             const float (&st_s)[2], bool adv) {
+  const uint64_t c2 = f2_pack(c[0], c[1]), s2 = f2_pack(s[0], s[1]);
+  const uint64_t tc2 = f2_pack(st_c[0], st_c[1]), ts2 = f2_pack(st_s[0], st_s[1]);
+  float nc[2], ns[2];
+  f2_unpack(f2_sub(f2_mul(c2, tc2), f2_mul(s2, ts2)), nc[0], nc[1]);
+  f2_unpack(f2_fma(c2, ts2, f2_mul(s2, tc2)), ns[0], ns[1]);
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    const float nc = c[e] * st_c[e] - s[e] * st_s[e];
-    const float ns = s[e] * st_c[e] + c[e] * st_s[e];
-    c[e] = adv ? nc : c[e];
-    s[e] = adv ? ns : s[e];
+    c[e] = adv ? nc[e] : c[e];
+    s[e] = adv ? ns[e] : s[e];
   }
 }
 
