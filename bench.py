@@ -85,7 +85,6 @@ def _source_hash(files):
 
 
 PREFILL_SRC = ["rope_context_extension_sm_b200/csrc/jl_prefill.cuh", "rope_context_extension_sm_b200/csrc/jl_device.cuh"]
-DECODE_SRC = ["rope_context_extension_sm_b200/csrc/jl_decode.cuh", "rope_context_extension_sm_b200/csrc/jl_device.cuh"]
 
 
 def _traffic(kernel, files):
