@@ -228,7 +228,10 @@ jl_status jl_bifocal_decode(const void* q, const void* k_cache, const void* v_ca
                             const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, jl_stream_t stream);
 
-/* Bytes of workspace jl_bifocal_decode / jl_plain_decode need for these sizes. */
+/* Bytes of workspace jl_bifocal_decode / jl_plain_decode need for these sizes,
+ * whatever the KV-head count: the split count depends on Hkv (as many splits as
+ * fit one wave of CTAs), so the size is the largest over every Hkv dividing Hq.
+ * 0 for non-positive sizes. */
 size_t jl_bifocal_decode_workspace_size(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen);
 
 /* Plain causal decode (no correction rotation), built from the same kernel;

@@ -22,14 +22,19 @@
 // CTA = one 128-row query block of one sequence x NQT query heads that share a
 // KV head (GQA).  Each K/V tile is loaded once by TMA and feeds all NQT heads.
 //   warp 0      TMA producer (Q, K, V tiles; 128B-swizzled boxes)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 4..   one warpgroup per query head: softmax on S read from TMEM,
-//               P written back to TMEM (bf16), O rescale, epilogue
-//   4 more      in-place RoPE rotation of the Q and K tiles in shared memory
-//   warps       (base rows R(x) or remote rows R(f(x))); each owns 32 rows and
-//               steps its cos/sin factors along the rows by complex
+//   warp 1      TMEM allocator + tcgen05.mma issuer (warp-uniform loop, one
+//               elected lane issues)
+//   warps 2, 3  in-place RoPE rotation of the Q and K tiles in shared memory
+//   and two     (base rows R(x) or remote rows R(f(x))); each owns 32 rows and
+//   more        steps its cos/sin factors along the rows by complex
 //               multiplication with e^{i theta_c}, anchored once per tile on a
 //               table row prefetched a tile ahead (no table load per row)
+//   warps 4..   one warpgroup per query head: the whole 128-column score row of
+//               each thread read from TMEM once per tile, softmax in registers,
+//               P written back to TMEM (bf16), O rescale, epilogue
+//   last two    idle (every warpgroup is complete for the register split)
+// Registers: launched at 65536 / threads per thread; setmaxnreg moves them from
+// the producer / MMA / rotation / idle warpgroups (56) to the softmax ones (200).
 // TMEM columns: S_t at 128 t, O_t at 128 NQT + D t; P_t aliases S_t.
 // With NQT = 2 the MMA issue order S0(n), PV1(n-1), S1(n), PV0(n) lets one
 // head's softmax overlap the other head's tensor-core work.

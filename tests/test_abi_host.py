@@ -97,6 +97,18 @@ def test_decode_workspace_size(jlmod):
     assert jlmod.jl_bifocal_decode_workspace_size(0, 32, 128, 131072) == 0
 
 
+@pytest.mark.parametrize("B,Hq,L", [(1, 32, 131072), (2, 32, 65536), (1, 16, 8192), (4, 64, 4096), (1, 8, 300)])
+def test_decode_workspace_covers_a_one_wave_split_for_every_kv_head_count(jlmod, B, Hq, L):
+    # The tensor-core decode runs at most one wave of 148 CTAs (B x Hkv x splits), each
+    # split a whole number of 128-key tiles; the size query does not know Hkv, so it has
+    # to cover the largest split any Hkv allowed by Hq can produce.
+    n = jlmod.jl_bifocal_decode_workspace_size(B, Hq, 128, L)
+    tiles = -(-L // 128)
+    for hkv in [h for h in range(1, Hq + 1) if Hq % h == 0 and Hq // h <= 16]:
+        worst_split = min(tiles, max(1, 148 // (hkv * B)))
+        assert n >= B * worst_split * Hq * (128 + 2) * 4, hkv
+
+
 def test_rope_tables_rejects_bad_arguments(jlmod):
     assert jlmod._lib.jl_rope_tables(16, 16, 0, 128, 1e4, None) == 1
     assert jlmod._lib.jl_rope_tables(16, 16, 10, 100, 1e4, None) == 2
