@@ -318,25 +318,58 @@ def run_ours(args, world, rank, local):
     jl.jl_sync_status()
 
     # ---- end to end through host buffers (H2D inputs, D2H outputs inside the timed region) ----
-    out_h = torch.empty_like(q_h).pin_memory()
-    lse_h = torch.empty((PREFILL.n_q_heads, L), dtype=torch.float32).pin_memory()
-    dout_h = torch.empty_like(dq_h).pin_memory()
-    e2e_steps = max(1, min(K, 3))
+    # Every step copies its inputs in from pinned host memory and its results out. The copies
+    # run on their own streams against double-buffered device tensors, so step s+1's inputs
+    # arrive and step s-1's results leave while step s computes; the timed region runs from
+    # the first input copy to the last result copy.
+    e2e_steps = max(2, K)
+    devbuf = [dict(q=q, k=k, v=v, dq=dq, out=out, lse=lse, dout=dout),
+              dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v), dq=torch.empty_like(dq),
+                   out=torch.empty_like(out), lse=torch.empty_like(lse), dout=torch.empty_like(dout))]
+    hostout = [dict(out=torch.empty_like(q_h).pin_memory(),
+                    lse=torch.empty((PREFILL.n_q_heads, L), dtype=torch.float32).pin_memory(),
+                    dout=torch.empty_like(dq_h).pin_memory()) for _ in range(2)]
+    h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
+
+    def copy_in(s_):
+        d = devbuf[s_ % 2]
+        with torch.cuda.stream(h2d_stream):
+            if s_ >= 2:
+                h2d_stream.wait_event(ev_done[s_ - 2])  # step s-2 has finished reading this buffer
+            for name, src in (("q", q_h), ("k", k_h), ("v", v_h), ("dq", dq_h)):
+                d[name].copy_(src, non_blocking=True)
+            ev_in[s_].record(h2d_stream)
+
     _barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(e2e_steps):
-        q.copy_(q_h, non_blocking=True)
-        k.copy_(k_h, non_blocking=True)
-        v.copy_(v_h, non_blocking=True)
-        dq.copy_(dq_h, non_blocking=True)
-        prefill()
-        decode()
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-        dout_h.copy_(dout, non_blocking=True)
+    h2d_stream.wait_event(a)
+    copy_in(0)
+    for s_ in range(e2e_steps):
+        d = devbuf[s_ % 2]
+        stream.wait_event(ev_in[s_])
+        if s_ >= 2:
+            stream.wait_event(ev_out[s_ - 2])  # step s-2's results have left this buffer
+        jl.jl_bifocal_prefill(d["q"], d["k"], d["v"], cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin,
+                              out=d["out"], lse=d["lse"])
+        jl.jl_bifocal_decode(d["dq"], dk, dv, dsl, DECODE_L, DECODE.w0, DECODE.w_pretrained, cos, sin,
+                             out=d["dout"], lse=dlse, workspace=dws)
+        ev_done[s_].record(stream)
+        if s_ + 1 < e2e_steps:
+            copy_in(s_ + 1)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ev_done[s_])
+            ho = hostout[s_ % 2]
+            for name in ("out", "lse", "dout"):
+                ho[name].copy_(d[name], non_blocking=True)
+            ev_out[s_].record(d2h_stream)
+    stream.wait_event(ev_out[e2e_steps - 1])
     b.record(stream)
     _barrier(world)
+    out_h, lse_h, dout_h = hostout[0]["out"], hostout[0]["lse"], hostout[0]["dout"]
     e2e_ms = _max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, dq_h))
     d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, dout_h))
