@@ -282,9 +282,30 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / n
 
+    def _time_graph(fns, reps):
+        """Device time per call of the calls in fns, captured once into a CUDA graph and replayed
+        reps times back to back (no host launch gaps between decode tokens)."""
+        for f in fns:  # once-per-process setup (kernel attributes) happens outside the capture
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / (reps * len(fns))
+
     plain_pre_ms = _time(plain_prefill, max(1, min(K, 3)))
-    plain_dec_ms = _time(plain_decode, 50)
-    bif_dec_ms_loop = _time(decode, 50)
+    plain_dec_ms = _time_graph([plain_decode], 200)
+    bif_dec_ms_loop = _time_graph([decode], 200)
 
     # ---- decode at the other cache lengths (rotating caches so each launch streams from HBM) ----
     sweep = {}
@@ -298,18 +319,18 @@ def run_ours(args, world, rank, local):
         sl = torch.tensor([Ld], dtype=torch.int32, device=dev)
         ws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, DECODE.n_q_heads, DECODE.head_dim, Ld),
                          dtype=torch.uint8, device=dev)
-        it = [0]
 
-        def dstep(plain=False):
-            kk, vv = caches[it[0] % n_rot]
-            it[0] += 1
+        def dstep(kk, vv, plain=False):
             if plain:
                 jl.jl_plain_decode(dq, kk, vv, sl, Ld, cos, sin, out=dout, lse=dlse, workspace=ws)
             else:
                 jl.jl_bifocal_decode(dq, kk, vv, sl, Ld, DECODE.w0, DECODE.w_pretrained, cos, sin, out=dout,
                                      lse=dlse, workspace=ws)
 
-        sweep[str(Ld)] = {"us": _time(dstep, 50) * 1e3, "plain_us": _time(lambda: dstep(True), 50) * 1e3,
+        reps = max(1, 200 // n_rot)
+        bif = [lambda kk=kk, vv=vv: dstep(kk, vv) for kk, vv in caches]
+        pln = [lambda kk=kk, vv=vv: dstep(kk, vv, True) for kk, vv in caches]
+        sweep[str(Ld)] = {"us": _time_graph(bif, reps) * 1e3, "plain_us": _time_graph(pln, reps) * 1e3,
                           "rotating_caches": n_rot}
         del caches
     for Ld, rec in sweep.items():

@@ -258,6 +258,46 @@ def test_small_decode_steps(jl, L):
     _check(out[0], lse[0], ro, rl, f"plain decode L={L}")
 
 
+def test_decode_replayed_from_a_cuda_graph_follows_the_device_lengths(jl):
+    # The decode entry point reads the lengths (and so G) only on the device, so one captured
+    # call serves every step: replaying it after the lengths change must give the eager result
+    # for the new lengths, bit for bit, crossing G = 4 -> 5 at L = 1024 -> 1025.
+    cfg = SMALL_DECODE
+    max_len = 1100
+    k_cache, v = _decode_setup(cfg, max_len)
+    kd, vd = k_cache.cuda(), v.cuda()
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    q_raw = I.decode_queries(cfg, 1)[0, 0]
+    sl = torch.tensor([1024], dtype=torch.int32, device="cuda")
+    qd = _query_tilde(cfg, q_raw, 1024)[None].cuda().contiguous()
+    out = torch.empty_like(qd)
+    lse = torch.empty((1, cfg.n_q_heads), dtype=torch.float32, device="cuda")
+    ws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, cfg.n_q_heads, cfg.head_dim, max_len),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        jl.jl_bifocal_decode(qd, kd, vd, sl, max_len, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse,
+                             workspace=ws)
+
+    step()  # one-time setup outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for L in (1024, 1025, 700):
+        sl.fill_(L)
+        qd.copy_(_query_tilde(cfg, q_raw, L)[None].cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        got_out, got_lse = out.clone(), lse.clone()
+        step()
+        jl.jl_sync_status()
+        assert torch.equal(got_out, out) and torch.equal(got_lse, lse), f"graph replay differs at L={L}"
+        ro, rl = _decode_oracle(cfg, _query_tilde(cfg, q_raw, L), k_cache[0], v[0], L)
+        _check(got_out.float().cpu().numpy()[0], got_lse.cpu().numpy()[0], ro, rl, f"graph decode L={L}")
+    del g
+
+
 def test_batched_decode_each_sequence_its_own_G(jl):
     cfg = SMALL_DECODE
     max_len, lens = 1024, [1024, 250, 513, 7]
