@@ -184,6 +184,104 @@ def replica_throughput(world, units_per_rank, steps, max_total_ms):
     return world * units_per_rank * steps / (max_total_ms * 1e-3)
 
 
+def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_ms, dk, dv, dq, dsl, dout, dlse,
+                       dws, dec_ms, hbm, sustained, _time, _time_graph):
+    """Device time of the rows built beyond the hot path, on the bench's own shapes.
+
+    - Literal three-pass prefill: the Qwen3-8B layer at L = 131072.
+    - KV-cache fill: the same layer's K/V into a base-RoPE cache.
+    - Decode append: one token.
+    - Chunked prefill: the last 8192 queries of the 131072-token sequence against the cache
+      of the first 122880 tokens plus the chunk.
+    - Paged decode: the 131072-token Qwen3-4B cache in 128-token pages in permuted order.
+    - Interpolation prefill: the remote pairs at scaled frequencies, lambda = 1/G.
+    """
+    L = PREFILL.seqlens[0]
+    d, hq, hkv = PREFILL.head_dim, PREFILL.n_q_heads, PREFILL.n_kv_heads
+    useful = PREFILL.useful_flops()
+    rows = {}
+
+    # literal inclusion-exclusion: three passes through the same kernel + the LSE merge
+    ws3 = torch.empty(3 * L * hq * d * 4 + 3 * L * hq * 4, dtype=torch.uint8, device=dev)
+    three = lambda: jl.jl_bifocal_prefill_three_pass(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin,
+                                                      out=out, lse=lse, workspace=ws3)
+    three()
+    ms = _time(three, 2)
+    rows["three_pass_prefill"] = {"ms": round(ms, 3), "useful_tflops": round(useful / (ms * 1e-3) / 1e12, 2),
+                                  "frac_of_bf16_peak_measured_sustained": round(useful / (ms * 1e-3) / 1e12 / sustained, 4),
+                                  "time_vs_fused": round(ms / fused_ms, 4)}
+    del ws3
+
+    # KV-cache fill: raw K, V -> R(j) k and v, one cache entry of L positions
+    kc = torch.empty((1, L, hkv, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    fill = lambda: jl.jl_kv_cache_fill(k, v, cu, cos, sin, kc, vc)
+    fill()
+    ms = _time(fill, 10)
+    fill_bytes = 4 * L * hkv * d * 2 + L * (d // 2) * 4 * 2  # K, V read + written, one table row pair per token
+    rows["kv_cache_fill"] = {"ms": round(ms, 4), "algorithmic_bytes": fill_bytes,
+                             "gbs": round(fill_bytes / (ms * 1e-3) / 1e9, 1),
+                             "frac_of_hbm_measured": round(fill_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+
+    # decode append: rotate one token's query, write its key and value (launch-bound)
+    sl1 = torch.tensor([L], dtype=torch.int32, device=dev)
+    q1 = q[:1].clone()
+    k1, v1 = k[:1].clone(), v[:1].clone()
+    q1_out = torch.empty_like(q1)
+    app = lambda: jl.jl_decode_append(q1, k1, v1, sl1, cos, sin, kc, vc, q_out=q1_out)
+    rows["decode_append"] = {"us": round(_time_graph([app], 200) * 1e3, 3)}
+
+    # chunked prefill: the last chunk of queries against the (filled) cache
+    chunk = 8192
+    past = L - chunk
+    qc = q[past:].contiguous()
+    cu_c = torch.tensor([0, chunk], dtype=torch.int32, device=dev)
+    past_t = torch.tensor([past], dtype=torch.int32, device=dev)
+    outc = torch.empty_like(qc)
+    lsec = torch.empty((hq, chunk), dtype=torch.float32, device=dev)
+    chk = lambda: jl.jl_bifocal_prefill_chunk(qc, cu_c, past_t, chunk, L, kc, vc, PREFILL.w0, PREFILL.w_pretrained,
+                                              cos, sin, out=outc, lse=lsec)
+    chk()
+    ms = _time(chk, 5)
+    chunk_flops = 4.0 * d * hq * sum(range(past + 1, L + 1))
+    rows["chunked_prefill"] = {"chunk": chunk, "past": past, "ms": round(ms, 3),
+                               "useful_tflops": round(chunk_flops / (ms * 1e-3) / 1e12, 2),
+                               "frac_of_bf16_peak_measured_sustained":
+                                   round(chunk_flops / (ms * 1e-3) / 1e12 / sustained, 4)}
+    del kc, vc, qc, outc
+
+    # paged decode: the decode cache as 128-token pages in a permuted pool
+    page = 128
+    n_pages = DECODE_L // page
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(7)).to(dev)
+    kp = torch.empty((n_pages, page, DECODE.n_kv_heads, DECODE.head_dim), dtype=torch.bfloat16, device=dev)
+    vp = torch.empty_like(kp)
+    kp[perm] = dk.view(n_pages, page, DECODE.n_kv_heads, DECODE.head_dim)
+    vp[perm] = dv.view(n_pages, page, DECODE.n_kv_heads, DECODE.head_dim)
+    table = perm.to(torch.int32).view(1, n_pages).contiguous()
+    pgd = lambda: jl.jl_bifocal_decode_paged(dq, kp, vp, table, dsl, DECODE_L, DECODE.w0, DECODE.w_pretrained, cos,
+                                             sin, out=dout, lse=dlse, workspace=dws)
+    us = _time_graph([pgd], 200) * 1e3
+    kv_bytes = 2 * DECODE_L * DECODE.n_kv_heads * DECODE.head_dim * 2
+    rows["paged_decode"] = {"page_size": page, "us_per_token": round(us, 2),
+                            "frac_of_hbm_measured": round(kv_bytes / (us * 1e-6) / 1e9 / hbm, 4),
+                            "time_vs_contiguous": round(us / (dec_ms * 1e3), 4)}
+    del kp, vp
+
+    # frequency-interpolation variant of the remote window (position interpolation, lambda = 1/G)
+    G = jl.jl_group_size(L, PREFILL.w_pretrained)
+    cr, sr = jl.jl_rope_tables_scaled(L, d, PREFILL.rope_base, [1.0 / G] * (d // 2), device=dev)
+    itp = lambda: jl.jl_interp_prefill(q, k, v, cu, L, PREFILL.w0, cos, sin, cr, sr, out=out, lse=lse)
+    itp()
+    ms = _time(itp, 2)
+    rows["interp_prefill"] = {"lambda": "1/G", "ms": round(ms, 3),
+                              "useful_tflops": round(useful / (ms * 1e-3) / 1e12, 2),
+                              "frac_of_bf16_peak_measured_sustained": round(useful / (ms * 1e-3) / 1e12 / sustained, 4),
+                              "time_vs_bifocal": round(ms / fused_ms, 4)}
+    del cr, sr
+    return rows
+
+
 # --------------------------------------------------------------- our arm ----
 
 def _build_decode_cache(L):
@@ -338,6 +436,11 @@ def run_ours(args, world, rank, local):
         rec["hbm_gbs"] = 2 * int(Ld) * DECODE.n_kv_heads * DECODE.head_dim * 2 / (rec["us"] * 1e-6) / 1e9
     jl.jl_sync_status()
 
+    # ---- rows beyond the hot path, each measured on its own workload ----
+    next_rows = _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, pre_avg, dk, dv, dq, dsl,
+                                   dout, dlse, dws, bif_dec_ms_loop, hbm, sustained, _time, _time_graph)
+    jl.jl_sync_status()
+
     # ---- end to end through host buffers (H2D inputs, D2H outputs inside the timed region) ----
     # Every step copies its inputs in from pinned host memory and its results out. The copies
     # run on their own streams against double-buffered device tensors, so step s+1's inputs
@@ -430,6 +533,7 @@ def run_ours(args, world, rank, local):
             "sweep": {k_: {kk: (round(vv, 3) if isinstance(vv, float) else vv) for kk, vv in r.items()}
                       for k_, r in sweep.items()},
         },
+        "next_rows": next_rows,
         "roofline": {
             "kernel": "jl_prefill_kernel<128,2>",
             "bound": "tensor",

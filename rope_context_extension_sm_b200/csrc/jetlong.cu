@@ -394,7 +394,8 @@ jl_status append_common(const void* q, const void* k, const void* v, const int32
   prm.max_pages = max_pages;
   prm.num_pages = num_pages;
   const int64_t rows = fill ? total_tokens * Hkv : static_cast<int64_t>(batch) * (Hq + Hkv);
-  const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  const int64_t warps = fill ? (rows + jl::kFillRowsPerWarp - 1) / jl::kFillRowsPerWarp : rows;
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
   if (fill) {
     if (head_dim == 128) jl::jl_kv_fill_kernel<128><<<blocks, 256, 0, st>>>(prm);
     else jl::jl_kv_fill_kernel<64><<<blocks, 256, 0, st>>>(prm);

@@ -7,8 +7,9 @@
 //
 // jl_kv_fill_kernel     prompt tokens (packed varlen) -> cache entries
 // jl_decode_append_kernel  one new token per entry: q~ = R(i) q, cache[i] = R(i) k, v
-// One warp per (token, head) row; lane l owns the rotate-half pairs (c, c + D/2)
-// for c in [l*D/64, l*D/64 + D/64), loads are coalesced row reads.
+// The fill kernel gives each warp four (token, head) rows, the append kernel one;
+// lanes own rotate-half pairs (c, c + D/2) and every access is a coalesced row read
+// or write.
 #pragma once
 
 #include "jl_device.cuh"
@@ -69,33 +70,92 @@ __device__ __forceinline__ void copy_row(const __nv_bfloat16* __restrict__ x, __
 }
 
 // Prompt tokens: token t of sequence b sits at position past[b] + t - cu_seqlens[b].
+// Each warp writes kFillRowsPerWarp consecutive (token, head) rows and issues all of
+// their loads (key words, table entries, value words) before the first store, so a
+// warp keeps several rows of DRAM reads in flight.  D = 128: lane l owns the
+// rotate-half pairs (2l, 64+2l) and (2l+1, 64+2l+1), read as two bf16x2 words, and
+// copies value channels 4l .. 4l+3 as one 8-byte word.  D = 64: lane l owns the pair
+// (l, l+32) and value channels 2l, 2l+1.
+constexpr int kFillRowsPerWarp = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
-  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;  // (token, head)
+  constexpr int R = kFillRowsPerWarp;
+  constexpr int HALF = D / 2;
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32 * R;
   const int lane = threadIdx.x & 31;
-  if (row >= p.total_tokens * p.Hkv) return;
-  const int64_t t = row / p.Hkv;
-  const int h = static_cast<int>(row % p.Hkv);
-  int lo = 0, hi = p.batch - 1;  // sequence holding token t: last b with cu[b] <= t
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.lens[mid] <= t) lo = mid; else hi = mid - 1;
+  const int64_t n_rows = p.total_tokens * p.Hkv;
+  int64_t src[R], dst[R], pos[R];
+  bool live[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {  // locate each row and check it against the cache
+    const int64_t row = row0 + r;
+    live[r] = row < n_rows;
+    src[r] = dst[r] = pos[r] = 0;
+    if (!live[r]) continue;
+    const int64_t t = row / p.Hkv;
+    const int h = static_cast<int>(row % p.Hkv);
+    int lo = 0, hi = p.batch - 1;  // sequence holding token t: last b with cu[b] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.lens[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    pos[r] = t - p.lens[b] + (p.past != nullptr ? p.past[b] : 0);
+    const int64_t crow = (pos[r] < 0 || pos[r] >= p.cache_stride || pos[r] >= p.n_tab_rows) ? -1
+                                                                                            : cache_row(p, b, pos[r]);
+    if (crow < 0) {
+      if (lane == 0) atomicOr(&g_status, kDevErrBounds);
+      live[r] = false;
+      continue;
+    }
+    src[r] = (t * p.Hkv + h) * D;
+    dst[r] = (crow * p.Hkv + h) * D;
   }
-  const int b = lo;
-  const int64_t pos = t - p.lens[b] + (p.past != nullptr ? p.past[b] : 0);
-  if (pos < 0 || pos >= p.cache_stride || pos >= p.n_tab_rows) {
-    if (lane == 0) atomicOr(&g_status, kDevErrBounds);
-    return;
+  if constexpr (D == 128) {
+    uint32_t ka[R], kb[R];
+    float2 cs[R], sn[R];
+    uint2 vw[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      ka[r] = *reinterpret_cast<const uint32_t*>(p.k + src[r] + 2 * lane);
+      kb[r] = *reinterpret_cast<const uint32_t*>(p.k + src[r] + HALF + 2 * lane);
+      cs[r] = *reinterpret_cast<const float2*>(p.cos_tab + pos[r] * HALF + 2 * lane);
+      sn[r] = *reinterpret_cast<const float2*>(p.sin_tab + pos[r] * HALF + 2 * lane);
+      vw[r] = *reinterpret_cast<const uint2*>(p.v + src[r] + 4 * lane);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ka[r]));
+      const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kb[r]));
+      const float2 ya = make_float2(a.x * cs[r].x - bb.x * sn[r].x, a.y * cs[r].y - bb.y * sn[r].y);
+      const float2 yb = make_float2(bb.x * cs[r].x + a.x * sn[r].x, bb.y * cs[r].y + a.y * sn[r].y);
+      *reinterpret_cast<__nv_bfloat162*>(p.k_cache + dst[r] + 2 * lane) = __float22bfloat162_rn(ya);
+      *reinterpret_cast<__nv_bfloat162*>(p.k_cache + dst[r] + HALF + 2 * lane) = __float22bfloat162_rn(yb);
+      *reinterpret_cast<uint2*>(p.v_cache + dst[r] + 4 * lane) = vw[r];
+    }
+  } else {
+    float ka[R], kb[R], cs[R], sn[R];
+    uint32_t vw[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      ka[r] = __bfloat162float(p.k[src[r] + lane]);
+      kb[r] = __bfloat162float(p.k[src[r] + HALF + lane]);
+      cs[r] = p.cos_tab[pos[r] * HALF + lane];
+      sn[r] = p.sin_tab[pos[r] * HALF + lane];
+      vw[r] = *reinterpret_cast<const uint32_t*>(p.v + src[r] + 2 * lane);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      p.k_cache[dst[r] + lane] = __float2bfloat16_rn(ka[r] * cs[r] - kb[r] * sn[r]);
+      p.k_cache[dst[r] + HALF + lane] = __float2bfloat16_rn(kb[r] * cs[r] + ka[r] * sn[r]);
+      *reinterpret_cast<uint32_t*>(p.v_cache + dst[r] + 2 * lane) = vw[r];
+    }
   }
-  const int64_t src = (t * p.Hkv + h) * D;
-  const int64_t crow = cache_row(p, b, pos);
-  if (crow < 0) {
-    if (lane == 0) atomicOr(&g_status, kDevErrBounds);
-    return;
-  }
-  const int64_t dst = (crow * p.Hkv + h) * D;
-  rotate_row_global<D>(p.k + src, p.k_cache + dst, pos, p, lane);
-  copy_row<D>(p.v + src, p.v_cache + dst, lane);
 }
 
 // One decode step: entry b's new token sits at i = seqlens[b] - 1.  Rows 0..Hq-1
