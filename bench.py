@@ -190,6 +190,7 @@ def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_m
 
     - Literal three-pass prefill: the Qwen3-8B layer at L = 131072.
     - KV-cache fill: the same layer's K/V into a base-RoPE cache.
+    - Prefill writing that cache itself (jl_bifocal_prefill_and_cache).
     - Decode append: one token.
     - Chunked prefill: the last 8192 queries of the 131072-token sequence against the cache
       of the first 122880 tokens plus the chunk.
@@ -222,6 +223,14 @@ def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_m
     rows["kv_cache_fill"] = {"ms": round(ms, 4), "algorithmic_bytes": fill_bytes,
                              "gbs": round(fill_bytes / (ms * 1e-3) / 1e9, 1),
                              "frac_of_hbm_measured": round(fill_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
+
+    # the same cache written by the prefill kernel itself, alongside the attention
+    pac = lambda: jl.jl_bifocal_prefill_and_cache(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin, kc, vc,
+                                                  out=out, lse=lse)
+    pac()
+    ms = _time(pac, 2)
+    rows["prefill_and_cache"] = {"ms": round(ms, 3), "useful_tflops": round(useful / (ms * 1e-3) / 1e12, 2),
+                                 "time_vs_prefill": round(ms / fused_ms, 4)}
 
     # decode append: rotate one token's query, write its key and value (launch-bound)
     sl1 = torch.tensor([L], dtype=torch.int32, device=dev)

@@ -141,6 +141,27 @@ jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const 
                              jl_stream_t stream);
 
 /*
+ * jl_bifocal_prefill that also writes the base-RoPE KV cache the decode reads
+ * (Methodology section 2: the cache holds the base keys R(j) k_j at their exact
+ * positions and is never rewritten afterwards).  The attention result equals
+ * jl_bifocal_prefill's; in addition, for every sequence b and position j:
+ *   k_cache[b][j][h] = bf16(R(j) k_j), v_cache[b][j][h] = v_j
+ *   k_cache, v_cache  bf16 [batch][cache_stride][Hkv][head_dim], caller-owned,
+ *                     16-byte aligned; positions >= the sequence length are not written
+ *   cache_stride      >= max_seqlen
+ * The kernel writes each key tile while it holds it rotated for its own query
+ * block (one CTA per KV head and block), so the cache costs no extra pass over K.
+ * w0 = 0 has no base-position visit when G > 1; then the cache is written by
+ * the cache-writer kernel (jl_kv_cache_fill) after the attention.
+ */
+jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                       int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq,
+                                       int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
+                                       const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                                       float softmax_scale, void* out, float* lse, void* k_cache, void* v_cache,
+                                       int64_t cache_stride, jl_stream_t stream);
+
+/*
  * Chunked prefill against a base-RoPE cache (a prompt processed in pieces, or
  * a long continuation of a conversation).  Entry b already holds past_lens[b]
  * keys/values in the caches, and this chunk's n_b = cu_seqlens[b+1] -

@@ -519,6 +519,37 @@ jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const 
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                       int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq,
+                                       int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
+                                       const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
+                                       float softmax_scale, void* out, float* lse, void* k_cache, void* v_cache,
+                                       int64_t cache_stride, jl_stream_t stream) {
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cache_stride < max_seqlen || cache_stride < 1)
+    return fail(JL_ERR_INVALID, "cache_stride (%lld) must be >= max_seqlen (%d) and >= 1", (long long)cache_stride,
+                max_seqlen);
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
+                               w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
+                               &empty);
+  if (s != JL_OK || empty) return s;
+  if (!k_cache || !v_cache) return fail(JL_ERR_INVALID, "null cache pointer");
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return fail(JL_ERR_INVALID, "caches must be 16-byte aligned");
+  prm.k_cache_out = static_cast<__nv_bfloat16*>(k_cache);
+  prm.v_cache_out = static_cast<__nv_bfloat16*>(v_cache);
+  prm.v_raw = static_cast<const __nv_bfloat16*>(v);
+  prm.cache_out_stride = cache_stride;
+  if ((s = launch_prefill_any(q, k, v, prm, head_dim, st)) != JL_OK) return s;
+  // With w0 = 0 and G > 1 no key tile is visited with base positions, so the kernel
+  // cannot write R(j) k_j; the cache writer fills the cache instead.
+  if (w0 == 0)
+    return append_common(nullptr, k, v, cu_seqlens, nullptr, batch, total_tokens, 0, Hkv, head_dim, cos_tab,
+                         sin_tab, n_tab_rows, nullptr, k_cache, v_cache, cache_stride, nullptr, 0, 0, 0, st, true);
+  return ok();
+}
+
 jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                            int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                            const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,

@@ -73,6 +73,12 @@ struct PrefillParams {
   int64_t n_rem_rows;
   const int32_t* past_lens;  // cached: tokens in each cache entry before this chunk
   int64_t cache_stride;      // cached: positions per cache entry
+  // Base-RoPE cache written by the prefill itself (NULL: not written): entry b, position j
+  // gets R(j) k_j and v_j; [batch][cache_out_stride][Hkv][D].  v_raw is the packed V input.
+  __nv_bfloat16* k_cache_out;
+  __nv_bfloat16* v_cache_out;
+  const __nv_bfloat16* v_raw;
+  int64_t cache_out_stride;
   float scale_log2;      // softmax scale * log2(e)
 };
 
@@ -324,6 +330,30 @@ __device__ __forceinline__ void correct_slice(uint8_t* tile, int rw, int kbase, 
         f.s[e] = cnt != 0 ? nf.s[e] : f.s[e];
       }
     }
+  }
+}
+
+// Copy rows [32 rw, 32 rw + 32) of a rotated 128-byte-swizzled K tile (shared
+// memory) and the same rows of raw V (global) to the cache rows of positions
+// pos0 + r of entry b, for r < n_valid.  16-byte chunks; consecutive lanes write
+// consecutive chunks of a row (D = 128: two rows per pass, D = 64: four).
+template <int D>
+__device__ __forceinline__ void write_cache_slice(const uint8_t* tile, int rw, const PrefillParams& p, int b,
+                                                  int pos0, int n_valid, int64_t v_tok0, int hkv, int lane) {
+  constexpr int kChunks = D / 8;          // 16-byte chunks per row
+  constexpr int kRowsPerPass = 32 / kChunks;
+  const int c = lane % kChunks;           // chunk of the row this lane copies
+  const int box = c >> 3, j = c & 7;      // 64-channel box and chunk inside its 128-byte row
+#pragma unroll 4
+  for (int r0 = 0; r0 < 32; r0 += kRowsPerPass) {
+    const int r = r0 + lane / kChunks;    // row within the slice
+    const int row = 32 * rw + r;          // row within the tile
+    if (row >= n_valid) continue;
+    const uint4 kw = *reinterpret_cast<const uint4*>(tile + box * 16384 + row * 128 + ((j ^ (row & 7)) << 4));
+    const int64_t dst = ((static_cast<int64_t>(b) * p.cache_out_stride + pos0 + row) * p.Hkv + hkv) * D + c * 8;
+    const int64_t src = ((v_tok0 + row) * p.Hkv + hkv) * D + c * 8;
+    *reinterpret_cast<uint4*>(p.k_cache_out + dst) = kw;
+    *reinterpret_cast<uint4*>(p.v_cache_out + dst) = *reinterpret_cast<const uint4*>(p.v_raw + src);
   }
 }
 
@@ -596,6 +626,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     };
     RotFactor<D> fk_next;
     load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
+    const bool write_cache = p.k_cache_out != nullptr && slot == 0 && p.mode == 0 && !p.cached;
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
       const bool rem_tab = interp && remote;  // interpolated rows at raw positions
@@ -617,6 +648,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
       if (!p.cached) {
         rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, stp, lane);
+        // The query block's own key tile, visited as local, now holds R(j) k_j: the first
+        // head slot of the KV group writes it (and the raw V rows) to the cache before the
+        // tile is released to the MMA, whose commit frees the stage.
+        if (write_cache && !remote && sc.kt(n) == qt) {
+          __syncwarp();
+          write_cache_slice<D>(sK + s * Lay::kTileBytes, rw, p, b, qt * kBN, n_rows - qt * kBN, q_tok0, hkv, lane);
+        }
       } else if (g > 1) {  // cached keys are base-rotated: local visits use them as they are
         switch (g) {
           case 2: correct_slice<D, 2>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, step, lane); break;

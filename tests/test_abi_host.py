@@ -109,6 +109,17 @@ def test_decode_workspace_covers_a_one_wave_split_for_every_kv_head_count(jlmod,
         assert n >= B * worst_split * Hq * (128 + 2) * 4, hkv
 
 
+def test_prefill_and_cache_rejects_a_short_cache_without_launching(jlmod):
+    lib = jlmod._lib
+    # cache_stride below max_seqlen is refused before any pointer is touched or kernel launched
+    st = lib.jl_bifocal_prefill_and_cache(None, None, None, None, 1, 100, 100, 4, 2, 128, 16, 64, None, None, 128,
+                                          0.0, None, None, None, None, 99, None)
+    assert st == 1 and "cache_stride" in jlmod.jl_last_error()
+    # an empty batch is a no-op, whatever the pointers
+    assert lib.jl_bifocal_prefill_and_cache(None, None, None, None, 0, 0, 0, 4, 2, 128, 16, 64, None, None, 1,
+                                            0.0, None, None, None, None, 1, None) == 0
+
+
 def test_rope_tables_rejects_bad_arguments(jlmod):
     assert jlmod._lib.jl_rope_tables(16, 16, 0, 128, 1e4, None) == 1
     assert jlmod._lib.jl_rope_tables(16, 16, 10, 100, 1e4, None) == 2

@@ -371,6 +371,42 @@ def test_kv_cache_fill_writes_base_rope_keys(jl):
         assert torch.count_nonzero(kc[b, L:]) == 0  # nothing written past the sequence
 
 
+PREFILL_AND_CACHE = [
+    ("varlen_G_to_10", (300, 1, 129, 0, 640), 4, 2, 128, 32, 64),
+    ("G1_plain", (200,), 4, 2, 128, 32, 256),
+    ("w0_0_writer_fallback", (300,), 4, 2, 128, 0, 64),
+    ("d64_group3", (257, 70), 3, 1, 64, 16, 64),
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_AND_CACHE, ids=[c[0] for c in PREFILL_AND_CACHE])
+def test_prefill_and_cache_writes_the_base_rope_cache(jl, case):
+    """Same attention as jl_bifocal_prefill, bit for bit; the cache holds R(p) k (one bf16
+    rounding of fp32 math) and v for every position of every sequence, nothing beyond."""
+    name, seqlens, hq, hkv, d, w0, w_pre = case
+    cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    stride = cfg.max_seqlen + 5
+    kc = torch.zeros((len(seqlens), stride, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    cos, sin = _tables(jl, stride, d, cfg.rope_base)
+    qd, kd, vd, cud = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
+    out, lse = jl.jl_bifocal_prefill_and_cache(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin, kc, vc)
+    ref_out, ref_lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin)
+    jl.jl_sync_status()
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    kc, vc = kc.cpu(), vc.cpu()
+    for b, L in enumerate(seqlens):
+        s0 = int(cu[b])
+        assert torch.count_nonzero(kc[b, L:]) == 0 and torch.count_nonzero(vc[b, L:]) == 0
+        if L == 0:
+            continue
+        pos = np.repeat(np.arange(L), hkv)
+        ref = O.rotate_rows(k[s0:s0 + L].float().numpy().reshape(-1, d), pos, cfg.rope_base).reshape(L, hkv, d)
+        np.testing.assert_allclose(kc[b, :L].float().numpy(), ref, rtol=2.0 ** -7, atol=1e-6)
+        assert torch.equal(vc[b, :L], v[s0:s0 + L])
+
+
 def test_cache_writer_reports_positions_outside_the_cache(jl):
     cos, sin = _tables(jl, 64, 128, 1e4)
     q = torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda")
