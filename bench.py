@@ -184,6 +184,75 @@ def replica_throughput(world, units_per_rank, steps, max_total_ms):
     return world * units_per_rank * steps / (max_total_ms * 1e-3)
 
 
+def _measure_other_configs(jl, dev, sustained, hbm, _time, _time_graph):
+    """The other workloads the metric is reported on, each on its own synthetic inputs.
+
+    - Qwen3-1.7B layer at L = 65536 (G = 2) for every w0 of the window sweep.
+    - The packed batch of 8 log-uniform sequences (4K-128K).
+    - A batched decode: 8 entries, cache lengths 8K-128K (each its own G), one token each.
+    """
+    res = {}
+    cfg = I.QWEN3_1P7B
+    q, k, v, cu = [t.to(dev) for t in I.prefill_inputs(cfg)]
+    L = cfg.seqlens[0]
+    cos, sin = jl.jl_rope_tables(L, cfg.head_dim, cfg.rope_base, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.n_q_heads, L), dtype=torch.float32, device=dev)
+    flops = cfg.useful_flops()
+    sweep = {}
+    for _ in range(10):  # ~0.2 s of the same work first, so every point runs at the steady-state clock
+        jl.jl_bifocal_prefill(q, k, v, cu, L, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+    for w0 in I.W0_SWEEP:
+        fn = lambda w0=w0: jl.jl_bifocal_prefill(q, k, v, cu, L, w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+        fn()
+        ms = _time(fn, 5)
+        sweep[str(w0)] = {"ms": round(ms, 3), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                          "frac_of_bf16_peak_measured_sustained": round(flops / (ms * 1e-3) / 1e12 / sustained, 4)}
+    pl = lambda: jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse)
+    pl()
+    ms = _time(pl, 5)
+    res["qwen3_1p7b_L65536_G2"] = {"w0_sweep": sweep, "plain_ms": round(ms, 3),
+                                   "plain_useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
+    del q, k, v, out, lse, cos, sin
+
+    cfg = I.VARLEN
+    q, k, v, cu = [t.to(dev) for t in I.prefill_inputs(cfg)]
+    mx = cfg.max_seqlen
+    cos, sin = jl.jl_rope_tables(mx, cfg.head_dim, cfg.rope_base, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.n_q_heads, q.shape[0]), dtype=torch.float32, device=dev)
+    flops = cfg.useful_flops()
+    fn = lambda: jl.jl_bifocal_prefill(q, k, v, cu, mx, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+    fn()
+    ms = _time(fn, 3)
+    res["varlen_8seq"] = {"seqlens": list(cfg.seqlens), "ms": round(ms, 3),
+                          "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                          "frac_of_bf16_peak_measured_sustained": round(flops / (ms * 1e-3) / 1e12 / sustained, 4)}
+    del q, k, v, out, lse
+
+    dc = DECODE
+    lens = [8192, 16384, 32768, 49152, 65536, 98304, 114688, 131072]
+    B, stride = len(lens), max(lens)
+    gen = torch.Generator(device=dev).manual_seed(11)  # timing-only inputs, drawn on the device
+    kc = torch.randn((B, stride, dc.n_kv_heads, dc.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    vc = torch.randn((B, stride, dc.n_kv_heads, dc.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    qd = torch.randn((B, dc.n_q_heads, dc.head_dim), generator=gen, device=dev).to(torch.bfloat16)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    dcos, dsin = jl.jl_rope_tables(stride, dc.head_dim, dc.rope_base, device=dev)
+    ws = torch.empty(jl.jl_bifocal_decode_workspace_size(B, dc.n_q_heads, dc.head_dim, stride), dtype=torch.uint8,
+                     device=dev)
+    dout = torch.empty_like(qd)
+    dlse = torch.empty((B, dc.n_q_heads), dtype=torch.float32, device=dev)
+    fn = lambda: jl.jl_bifocal_decode(qd, kc, vc, sl, stride, dc.w0, dc.w_pretrained, dcos, dsin, out=dout, lse=dlse,
+                                      workspace=ws)
+    us = _time_graph([fn], 100) * 1e3
+    kv_bytes = sum(2 * Lb * dc.n_kv_heads * dc.head_dim * 2 for Lb in lens)
+    res["batched_decode_8"] = {"cache_lens": lens, "us_per_step": round(us, 2),
+                               "hbm_gbs": round(kv_bytes / (us * 1e-6) / 1e9, 1),
+                               "frac_of_hbm_measured": round(kv_bytes / (us * 1e-6) / 1e9 / hbm, 4)}
+    return res
+
+
 def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_ms, dk, dv, dq, dsl, dout, dlse,
                        dws, dec_ms, hbm, sustained, _time, _time_graph):
     """Device time of the rows built beyond the hot path, on the bench's own shapes.
@@ -449,6 +518,8 @@ def run_ours(args, world, rank, local):
     next_rows = _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, pre_avg, dk, dv, dq, dsl,
                                    dout, dlse, dws, bif_dec_ms_loop, hbm, sustained, _time, _time_graph)
     jl.jl_sync_status()
+    other_configs = _measure_other_configs(jl, dev, sustained, hbm, _time, _time_graph)
+    jl.jl_sync_status()
 
     # ---- end to end through host buffers (H2D inputs, D2H outputs inside the timed region) ----
     # Every step copies its inputs in from pinned host memory and its results out. The copies
@@ -543,6 +614,7 @@ def run_ours(args, world, rank, local):
                       for k_, r in sweep.items()},
         },
         "next_rows": next_rows,
+        "other_configs": other_configs,
         "roofline": {
             "kernel": "jl_prefill_kernel<128,2>",
             "bound": "tensor",

@@ -202,8 +202,12 @@ bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) { return head_dim
 // Keys per split.  CUDA-core kernel: a power of two in [64, 512].  Tensor-core
 // kernel: whole 128-key tiles, as many splits per (entry, KV head) as fit the
 // 148 SMs of a B200 in ONE wave (one CTA per SM): a CTA left over for a second
-// wave would run after all the others and set the kernel's time.
+// wave would run after all the others and set the kernel's time.  When one wave
+// would leave each CTA more than kMaxTilesPerSplit tiles to walk (many entries x
+// KV heads), the splits are cut to that length instead and the grid runs in
+// several waves; splits past an entry's length exit at once.
 constexpr int64_t kSMs = 148;
+constexpr int64_t kMaxTilesPerSplit = 128;
 
 int chunk_cuda_core(int32_t max_seqlen) {
   int c = 64;
@@ -215,7 +219,7 @@ int chunk_tc(int32_t B, int32_t Hkv, int32_t max_seqlen) {
   const int64_t tiles = (static_cast<int64_t>(max_seqlen) + jl::kDecTile - 1) / jl::kDecTile;
   const int64_t ctas_per_split = static_cast<int64_t>(Hkv) * B;
   const int64_t n_target = std::max<int64_t>(1, kSMs / std::max<int64_t>(1, ctas_per_split));
-  const int64_t per = std::max<int64_t>(1, (tiles + n_target - 1) / n_target);
+  const int64_t per = std::min(kMaxTilesPerSplit, std::max<int64_t>(1, (tiles + n_target - 1) / n_target));
   return static_cast<int>(per * jl::kDecTile);
 }
 
