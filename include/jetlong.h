@@ -3,9 +3,11 @@
  * on NVIDIA B200 (sm_100a).
  *
  * Method: "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
- * RoPE" (Tang, Wang, Gu, Han, Cai, 2026), as summarised on the web pages
- * gist.science/es, gist.science/de and gist.science/ja (Methodology sections
- * 1 and 2) and in the abstract on chatpaper.ai/fr.
+ * RoPE" (Tang, Wang, Gu, Han, Cai, 2026), as summarised on the pages
+ * "Resumen Técnico: Jet-Long", "Jet-Long: Efficient Long-Context Extension with
+ * Dynamic Bifocal RoPE" and "技術要約: Jet-Long" (Methodology sections 1 and 2)
+ * and in the abstract of "Jet-Long : Extension efficace de long contexte avec
+ * RoPE bifocale dynamique".
  *
  * Notation.  L: length of a sequence (prefill) or of the cache including the
  * current token (decode).  w_pretrained: pretraining window.  w0: local window.

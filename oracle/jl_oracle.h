@@ -8,8 +8,10 @@
  * value produced by the CUDA library.
  *
  * Sources (the paper "Jet-Long: Efficient Long-Context Extension with Dynamic
- * Bifocal RoPE", Tang, Wang, Gu, Han, Cai, 2026, as summarised on the web pages
- * gist.science/es, gist.science/de, gist.science/ja and chatpaper.ai/fr):
+ * Bifocal RoPE", Tang, Wang, Gu, Han, Cai, 2026, as summarised on the pages
+ * "Resumen Técnico: Jet-Long", "Jet-Long: Efficient Long-Context Extension with
+ * Dynamic Bifocal RoPE", "技術要約: Jet-Long" and "Jet-Long : Extension efficace
+ * de long contexte avec RoPE bifocale dynamique"):
  *   - Methodology, section 1 "Dynamic Bifocal RoPE": the local window of w0
  *     keeps classical RoPE; positions beyond it use the remote map
  *     f(x) = floor(x / G) with G = max(1, ceil(L / w_pretrained)).
