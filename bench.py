@@ -360,6 +360,71 @@ def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_m
     return rows
 
 
+def _measure_walk(jl, dev, stream, dk, dv, cos, sin):
+    """The generation walk of the decode workload: 256 tokens at query positions 98176 .. 98431,
+    crossing L = 98304 -> 98305 where G goes from 3 to 4.  Each step appends the token (its query
+    rotated to R(i) q, its key rotated into the base-RoPE cache, its value stored) and decodes it
+    against the cache with the correction rotation on the fly.  Every step is timed on the device
+    with its own pair of CUDA events; the same walk through the plain decode is the comparator.
+    The tokens' q/k/v are seeded random bf16; the cache rows before the walk are the bench's."""
+    first, steps = DECODE.walk_first_pos, DECODE.walk_steps
+    max_len = first + steps
+    hq, hkv, d = DECODE.n_q_heads, DECODE.n_kv_heads, DECODE.head_dim
+    gen = torch.Generator(device=dev).manual_seed(5)
+    wq = torch.randn((steps, 1, hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    wk = torch.randn((steps, 1, hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    wv = torch.randn((steps, 1, hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    sls = torch.arange(first + 1, first + steps + 1, dtype=torch.int32, device=dev).view(steps, 1)
+    qt = torch.empty((1, hq, d), dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(qt)
+    lse = torch.empty((1, hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, hq, d, max_len), dtype=torch.uint8, device=dev)
+
+    def step(t, plain):
+        jl.jl_decode_append(wq[t], wk[t], wv[t], sls[t], cos, sin, dk, dv, q_out=qt)
+        if plain:
+            jl.jl_plain_decode(qt, dk, dv, sls[t], max_len, cos, sin, out=out, lse=lse, workspace=ws)
+        else:
+            jl.jl_bifocal_decode(qt, dk, dv, sls[t], max_len, DECODE.w0, DECODE.w_pretrained, cos, sin, out=out,
+                                 lse=lse, workspace=ws)
+
+    def walk(plain):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(stream)
+        for t in range(steps):
+            step(t, plain)
+            ev[t + 1].record(stream)
+        torch.cuda.synchronize()
+        return [ev[t].elapsed_time(ev[t + 1]) * 1e3 for t in range(steps)]
+
+    walk(False)  # warm: every launch shape of the walk once
+    walk(True)
+    bif, pln = walk(False), walk(True)
+    jl.jl_sync_status()
+    Ls = [first + t + 1 for t in range(steps)]
+    before = [t for t in range(steps) if jl.jl_group_size(Ls[t], DECODE.w_pretrained) == 3]
+    after = [t for t in range(steps) if jl.jl_group_size(Ls[t], DECODE.w_pretrained) == 4]
+
+    def stats(xs):
+        return {"min": round(min(xs), 2), "median": round(statistics.median(xs), 2), "max": round(max(xs), 2)}
+
+    def side(ts):
+        b, p = [bif[t] for t in ts], [pln[t] for t in ts]
+        return {"steps": len(ts), "L": [Ls[ts[0]], Ls[ts[-1]]], "us_per_token": stats(b), "plain_us_per_token": stats(p),
+                "overhead_vs_plain": round(statistics.median(b) / statistics.median(p) - 1.0, 4)}
+
+    boundary = Ls.index(first + 128)  # the last step at G = 3 (L = 98304) and the first at G = 4
+    return {
+        "tokens": steps, "query_positions": [first, first + steps - 1], "G": [3, 4],
+        "step": "jl_decode_append + jl_bifocal_decode (plain: jl_decode_append + jl_plain_decode)",
+        "us_per_token": stats(bif), "plain_us_per_token": stats(pln),
+        "overhead_vs_plain": round(statistics.median(bif) / statistics.median(pln) - 1.0, 4),
+        "G3_side": side(before), "G4_side": side(after),
+        "around_boundary_us": {str(Ls[t]): round(bif[t], 2) for t in range(boundary - 2, boundary + 3)},
+        "plain_around_boundary_us": {str(Ls[t]): round(pln[t], 2) for t in range(boundary - 2, boundary + 3)},
+    }
+
+
 # --------------------------------------------------------------- our arm ----
 
 def _build_decode_cache(L):
@@ -514,6 +579,9 @@ def run_ours(args, world, rank, local):
         rec["hbm_gbs"] = 2 * int(Ld) * DECODE.n_kv_heads * DECODE.head_dim * 2 / (rec["us"] * 1e-6) / 1e9
     jl.jl_sync_status()
 
+    # ---- the 256-token generation walk across the G = 3 -> 4 boundary ----
+    decode_walk = _measure_walk(jl, dev, stream, dk, dv, cos, sin)
+
     # ---- rows beyond the hot path, each measured on its own workload ----
     next_rows = _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, pre_avg, dk, dv, dq, dsl,
                                    dout, dlse, dws, bif_dec_ms_loop, hbm, sustained, _time, _time_graph)
@@ -601,6 +669,13 @@ def run_ours(args, world, rank, local):
             "plain_ms": round(plain_pre_ms, 4),
             "plain_useful_tflops": round(flops / (plain_pre_ms * 1e-3) / 1e12, 2),
             "bifocal_over_plain_time": round(pre_avg / plain_pre_ms, 4),
+            # clock-normalised: useful flops per SM cycle at the median SM clock of the timed region,
+            # against the tensor pipe's 8192 dense bf16 flops per SM cycle
+            "sm_mhz_median": clocks["sm_mhz"] if clocks else None,
+            "useful_flop_per_sm_cycle": (round(flops / (pre_avg * 1e-3 * clocks["sm_mhz"] * 1e6 * 148), 1)
+                                         if clocks else None),
+            "tensor_frac_at_measured_clock": (round(flops / (pre_avg * 1e-3 * clocks["sm_mhz"] * 1e6 * 148) / 8192, 4)
+                                              if clocks else None),
         },
         "decode": {
             # back-to-back tokens: one decode call captured in a CUDA graph, replayed 200 times
@@ -616,6 +691,7 @@ def run_ours(args, world, rank, local):
             "overhead_vs_plain": round(bif_dec_ms_loop / plain_dec_ms - 1.0, 4),
             "sweep": {k_: {kk: (round(vv, 3) if isinstance(vv, float) else vv) for kk, vv in r.items()}
                       for k_, r in sweep.items()},
+            "walk": decode_walk,
         },
         "next_rows": next_rows,
         "other_configs": other_configs,
@@ -647,18 +723,17 @@ def run_ours(args, world, rank, local):
 
 # ----------------------------------------------------- CPU oracle (baseline) ----
 
-def _oracle_sample_rows(n_rows, seed=7):
-    rng = np.random.default_rng(seed)
-    L = PREFILL.seqlens[0]
-    pos = rng.integers(L // 2, L, n_rows)
-    head = rng.integers(0, PREFILL.n_q_heads, n_rows)
-    return pos, head
+def _host_cores():
+    """Cores this process may run on (affinity-aware nproc)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
 
 
-def cpu_baseline(seconds=15.0, inputs=None):
-    """The fp64 oracle as it stands, on a bounded sample of the prefill workload: rows drawn
-    uniformly from the second half of the 128K sequence, all query heads of KV head 0."""
-    from oracle import oracle as O
+def _cpu_prefill_rows(O, seconds, inputs=None):
+    """The fp64 oracle on rows drawn uniformly from the second half of the 128K sequence, all
+    query heads of KV head 0, for about `seconds` of oracle time."""
     if inputs is None:
         q_h, k_h, v_h, _ = I.prefill_inputs(PREFILL)
     else:
@@ -679,27 +754,87 @@ def cpu_baseline(seconds=15.0, inputs=None):
         done_rows += n
         done_flops += float(np.sum(4.0 * PREFILL.head_dim * (pos + 1)))
         n = min(n * 2, 256)
+    return done_rows, done_flops, spent
+
+
+def _cpu_decode(O):
+    """The oracle's decode step (fp64) on the decode workload: one step at each cache length, and
+    the four steps of the 256-token walk on either side of the G = 3 -> 4 boundary (L = 98303 ..
+    98306).  The whole walk is extrapolated from those four and labelled an estimate."""
+    cfg = DECODE
+    first, steps = cfg.walk_first_pos, cfg.walk_steps
+    max_len = max(max(cfg.cache_lens), first + steps)
+    k_raw, v = I.decode_raw_inputs(cfg, max_len)  # random rows stand for base-rotated keys
+    kb, vb = I.bf16_bits(k_raw[0]), I.bf16_bits(v[0])
+    qb = I.bf16_bits(I.decode_queries(cfg, 1)[0, 0])
+
+    def one(L):
+        t0 = time.perf_counter()
+        O.decode_step(qb, kb[:L], vb[:L], L, w0=cfg.w0, w_pretrained=cfg.w_pretrained, rope_base=cfg.rope_base)
+        return time.perf_counter() - t0
+
+    per_len = {str(L): round(one(L) * 1e6, 1) for L in cfg.cache_lens}
+    walk_L = [first + 127, first + 128, first + 129, first + 130]
+    walk_s = [one(L) for L in walk_L]
     return {
+        "unit": "us/token",
+        "us_per_token_at_cache_len": per_len,
+        "walk_sample": {"L": walk_L, "G": [O.group_size(L, cfg.w_pretrained) for L in walk_L],
+                        "us_per_token": [round(t * 1e6, 1) for t in walk_s]},
+        "walk_256_tokens_estimate_s": round(statistics.mean(walk_s) * steps, 2),
+    }
+
+
+def _cpu_tiny(O):
+    """Config 1 (L = 256, one head, head_dim 64, G = 4, w0 = 32) in full: every row."""
+    cfg = I.TINY
+    q, k, v, _ = I.prefill_inputs(cfg)
+    L = cfg.seqlens[0]
+    qb, kb, vb = I.bf16_bits(q), I.bf16_bits(k), I.bf16_bits(v)
+    pos, head = np.arange(L), np.zeros(L, dtype=np.int64)
+    reps, t0 = 0, time.perf_counter()
+    while reps < 3 or time.perf_counter() - t0 < 0.5:
+        O.bifocal_rows(qb, kb, vb, L, pos, head, w0=cfg.w0, w_pretrained=cfg.w_pretrained, rope_base=cfg.rope_base)
+        reps += 1
+    dt = (time.perf_counter() - t0) / reps
+    return {"ms_per_layer": round(dt * 1e3, 3), "useful_tflops": cfg.useful_flops() / dt / 1e12,
+            "sample": f"the whole tiny layer ({L} rows), mean of {reps} runs"}
+
+
+def cpu_baseline(seconds=15.0, inputs=None, with_decode=True):
+    """The fp64 oracle as it stands, timed on the host cores: a bounded sample of the 128K prefill
+    (the headline metric's unit), plus the decode step and the tiny layer."""
+    from oracle import oracle as O
+    done_rows, done_flops, spent = _cpu_prefill_rows(O, seconds, inputs)
+    res = {
         "value": done_flops / spent / 1e12,
         "unit": UNIT,
-        "cores": O.num_threads(),
+        "cores": _host_cores(),
+        "omp_threads": O.num_threads(),
         "kind": "oracle",
         "sample": f"{done_rows} query rows of the L=131072 prefill (positions in [65536, 131072), KV head 0), "
                   f"{spent:.1f} s; useful flops of those rows / time",
         "full_layer_estimate_s": PREFILL.useful_flops() / (done_flops / spent),
     }
+    if with_decode:
+        res["decode"] = _cpu_decode(O)
+        res["tiny"] = _cpu_tiny(O)
+    return res
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    from oracle import oracle as O
     q_h, k_h, v_h, _ = I.prefill_inputs(PREFILL)
     inputs = (q_h, k_h, v_h)
     for _ in range(args.warmup):
-        cpu_baseline(seconds=0.5, inputs=inputs)
+        cpu_baseline(seconds=0.5, inputs=inputs, with_decode=False)
     per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps)))
-    vals = [cpu_baseline(seconds=per_step, inputs=inputs) for _ in range(args.steps)]
+    vals, step_s = [], []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        vals.append(cpu_baseline(seconds=per_step, inputs=inputs, with_decode=False))
+        step_s.append(time.perf_counter() - t0)
     v = statistics.mean(r["value"] for r in vals)
     return {
         "impl": "reference",
@@ -709,15 +844,15 @@ def run_reference(args, world, rank):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": per_step * 1e3,
+        "ms_per_step": statistics.mean(step_s) * 1e3,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16, outlier-scaled key channels)",
         "config": _config(),
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle",
-                         "sample": vals[0]["sample"]},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"], "omp_threads": vals[0]["omp_threads"],
+                         "kind": "oracle", "sample": vals[0]["sample"] + f"; each step a sample of {per_step:.0f} s"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -67,6 +67,18 @@ int64_t jl_group_size(int64_t L, int64_t w_pretrained);
 jl_status jl_sync_status(jl_stream_t stream);
 
 /*
+ * Debug-bounds build (no counterpart in the paper; a diagnostic of this library).
+ * Returns 1 in the library built with -DJL_DEBUG_BOUNDS (libjetlong_bounds.so),
+ * 0 otherwise.  That build checks on the device every index its kernels derive
+ * there -- RoPE table rows (remote rows < w_pretrained, every row < n_tab_rows),
+ * TMA tile coordinates against the sequence or cache they belong to, cache and
+ * page positions, workspace slots -- and records a failed check in the status
+ * word instead of trapping; jl_sync_status() then returns JL_ERR_INVALID.  The
+ * checks are compiled out of the normal build.
+ */
+int jl_debug_bounds_enabled(void);
+
+/*
  * Failure-detection self-test (no counterpart in the paper; it exercises this
  * library's bounded waits).  Launches one thread that waits on a shared-memory
  * barrier that nothing ever completes, giving up after limit_cycles SM clock
@@ -79,7 +91,10 @@ jl_status jl_sync_status(jl_stream_t stream);
 jl_status jl_selftest_wait_timeout(int64_t limit_cycles, jl_stream_t stream);
 
 /*
- * RoPE cos/sin tables.  Fills cos_out[p][c] = cos(p * theta_c) and
+ * RoPE cos/sin tables (Methodology section 1, "Dynamic Bifocal RoPE": the local
+ * window keeps classical RoPE at the true positions, and positions beyond it
+ * are rotated at the remote positions f(x); both rotations are rows of this one
+ * table).  Fills cos_out[p][c] = cos(p * theta_c) and
  * sin_out[p][c] = sin(p * theta_c) for p in [0, n_pos), c in [0, head_dim/2),
  * row-major fp32 [n_pos][head_dim/2].  Angles and cos/sin are computed in fp64
  * on the device and rounded to fp32 once.  Both the base rotations R(i) and the
@@ -244,6 +259,8 @@ jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const in
  * (R(f(i) - i) q) . (R(f(j) - j) k_cache[j]), both corrections applied in
  * registers.  G = max(1, ceil(seqlens[b] / w_pretrained)) is computed on the
  * device every call.
+ * Supported: head_dim 128 (tensor cores) or 64 (CUDA cores), 1 to 16 query
+ * heads per KV head; more returns JL_ERR_UNSUPPORTED.
  */
 jl_status jl_bifocal_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
                             int32_t B, int64_t cache_stride, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
@@ -339,9 +356,14 @@ jl_status jl_decode_append_paged(const void* q, const void* k, const void* v, co
  *    (head_dim + 2) * 4 bytes, see jl_bifocal_decode_workspace_size) return
  *    JL_ERR_INVALID with a message; B = 1, Hq = 32, head_dim = 128 fits up to
  *    max_seqlen = 131072.
- *  - The first call on a device looks up the array's device address (the
- *    device current at the call is the one used); make that first call before
- *    any stream capture.
+ *  - The stream, the current device and q must be on one device; a mismatch
+ *    returns JL_ERR_INVALID (the array's address is only valid on its own
+ *    device).  Each call outside stream capture looks the address up again with
+ *    cudaGetSymbolAddress, so a reset device context is picked up; a call made
+ *    during a capture uses the address from the last uncaptured call on that
+ *    device, so make the first call on a device before any stream capture.
+ *  - If a kernel of the call gives up on a bounded wait (jl_sync_status then
+ *    reports JL_ERR_TIMEOUT), out and lse are written as NaN.
  *  - All calls on a device share the one array, and it keeps whatever the last
  *    call left there (nothing in it needs to start at zero).  Calls whose
  *    executions overlap on the GPU -- on different streams, or from different

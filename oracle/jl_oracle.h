@@ -20,7 +20,7 @@
  *     inclusion-exclusion merge of three flash-style passes on LogSumExp
  *     statistics, which yields the exact distance-routed output.
  *
- * Readings of points the pages leave open (each is repeated in the design doc):
+ * Readings of points the pages leave open:
  *   C1 local  <=>  0 <= i - j < w0   (distance, strict; w0 keys incl. self)
  *   C2 the remote score rotates the query by f(i) and the key by f(j)
  *   C3 positions are 0-based per sequence; L is the sequence length (prefill)

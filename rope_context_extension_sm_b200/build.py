@@ -31,16 +31,27 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*")) + [os.path.join(ROOT, "include", "jetlong.h")])
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+# The debug-bounds build: the same library with device-side index checks compiled in
+# (-DJL_DEBUG_BOUNDS; each failed check is recorded in the status word, see jl_device.cuh).
+BOUNDS_LIB = os.path.join(HERE, "libjetlong_bounds.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, out: str | None = None) -> str:
+    out = out or LIB
     newest = max(os.path.getmtime(p) for p in sources())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not extra:
-        return LIB
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest and (not extra or out != LIB):
+        return out
     cmd = [NVCC, *FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           "-o", LIB, os.path.join(CSRC, "jetlong.cu")]
+           "-o", out, os.path.join(CSRC, "jetlong.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    return LIB
+    return out
+
+
+def build_bounds(force: bool = False) -> str:
+    """Build libjetlong_bounds.so (the debug-bounds variant) in-tree."""
+    return build(force=force, extra=["-DJL_DEBUG_BOUNDS"], out=BOUNDS_LIB)
 
 
 if __name__ == "__main__":

@@ -10,8 +10,10 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "jetlong.h"
 #include "jl_append.cuh"
@@ -46,6 +48,39 @@ jl_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// ------------------------------------------------------ kernel attributes --
+//
+// Function attributes (the dynamic shared-memory limit) belong to the device
+// context a launch runs in, so the one-time setting is kept per (device,
+// kernel): a process that drives a second GPU sets it there too.  A failed
+// attempt is not remembered, so the next launch tries again.
+
+struct KernelAttr {
+  cudaError_t err;
+  int regs;  // registers per thread of the built kernel
+};
+
+std::mutex g_attr_mu;
+std::map<std::pair<int, const void*>, KernelAttr> g_attr;
+
+KernelAttr kernel_attr(const void* kern, int smem_bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return {e, 0};
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  const auto key = std::make_pair(dev, kern);
+  const auto it = g_attr.find(key);
+  if (it != g_attr.end()) return it->second;
+  KernelAttr a{cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes), 0};
+  if (a.err == cudaSuccess) {
+    cudaFuncAttributes fa{};
+    a.err = cudaFuncGetAttributes(&fa, kern);
+    a.regs = fa.numRegs;
+  }
+  if (a.err == cudaSuccess) g_attr[key] = a;
+  return a;
+}
+
 // ---------------------------------------------------------------- TMA maps --
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -76,6 +111,25 @@ jl_status make_map(CUtensorMap* map, const void* base, int64_t tokens, int heads
   return JL_OK;
 }
 
+// Launch with the programmatic stream-serialization attribute: the kernel may be
+// scheduled while the previous kernel of the stream still runs, and waits for it
+// in griddep_wait() (jl_device.cuh) before touching its results.  This hides the
+// launch latency of the short decode kernels behind the kernel before them.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ----------------------------------------------------------------- prefill --
 
 template <int D, int NQT>
@@ -90,16 +144,9 @@ jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::
   if ((s = make_map(&tk, k, kv_rows, prm.Hkv, D)) != JL_OK) return s;
   if ((s = make_map(&tv, v, kv_rows, prm.Hkv, D)) != JL_OK) return s;
   auto kern = jl::jl_prefill_kernel<D, NQT>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  static int launch_regs = 0;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
-    cudaFuncAttributes fa{};
-    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, kern);
-    launch_regs = fa.numRegs;
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(prefill)");
+  const KernelAttr attr = kernel_attr(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+  if (attr.err != cudaSuccess) return cuda_fail(attr.err, "cudaFuncSetAttribute(prefill)");
+  const int launch_regs = attr.regs;
   // The kernel moves registers between its warpgroups (setmaxnreg); the softmax
   // warpgroups' increase would wait forever if the launch allocation could not
   // cover the split, so such a build is refused here rather than launched.
@@ -194,10 +241,15 @@ size_t three_pass_ws_bytes(int64_t total_tokens, int32_t Hq, int32_t head_dim) {
 
 // ------------------------------------------------------------------ decode --
 
-// Tensor-core decode (head_dim 128, up to 16 query heads per KV head) splits the
-// keys in chunks of whole 128-key tiles, sized for one wave of CTAs; the other
-// shapes use the CUDA-core split kernel.
-bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) { return head_dim == 128 && Hq / Hkv <= 16; }
+// Tensor-core decode (head_dim 128) splits the keys in chunks of whole 128-key
+// tiles, sized for one wave of CTAs; head_dim 64 uses the CUDA-core split kernel.
+// Both take up to 16 query heads per KV head: each is built for the group
+// capacities 1, 2, 4, 8 and 16, and a group in between runs in the next capacity
+// up with the spare query rows held at zero.
+constexpr int32_t kMaxDecodeGroup = 16;
+bool decode_uses_tc(int32_t head_dim, int32_t Hq, int32_t Hkv) {
+  return head_dim == 128 && Hq / Hkv <= kMaxDecodeGroup;
+}
 
 // Keys per split.  CUDA-core kernel: a power of two in [64, 512].  Tensor-core
 // kernel: whole 128-key tiles, as many splits per (entry, KV head) as fit the
@@ -233,18 +285,12 @@ jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) 
   if ((s = make_map(&tk, prm.k, rows, prm.Hkv, 128)) != JL_OK) return s;
   if ((s = make_map(&tv, prm.v, rows, prm.Hkv, 128)) != JL_OK) return s;
   auto kern = jl::jl_decode_tc_kernel<GROUP, PLAIN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(decode)");
+  const KernelAttr attr = kernel_attr(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+  if (attr.err != cudaSuccess) return cuda_fail(attr.err, "cudaFuncSetAttribute(decode)");
   dim3 grid(prm.Hkv, prm.n_split, B);
-  kern<<<grid, Lay::kThreads, Lay::kAlloc, st>>>(tk, tv, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, grid, dim3(Lay::kThreads), Lay::kAlloc, st, tk, tv, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  jl::jl_decode_combine_kernel<128><<<dim3(prm.Hq, B), jl::kCombineThreads, 0, st>>>(prm);
-  e = cudaGetLastError();
+  e = launch_pdl(jl::jl_decode_combine_kernel<128>, dim3(prm.Hq, B), dim3(jl::kCombineThreads), 0, st, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return ok();
 }
@@ -252,33 +298,30 @@ jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) 
 template <int D, int GROUP, bool PLAIN>
 jl_status launch_decode(const jl::DecodeParams& prm, int B, cudaStream_t st) {
   dim3 grid(prm.Hkv, prm.n_split, B);
-  jl::jl_decode_split_kernel<D, GROUP, PLAIN><<<grid, jl::kDecodeThreads, 0, st>>>(prm);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(jl::jl_decode_split_kernel<D, GROUP, PLAIN>, grid, dim3(jl::kDecodeThreads), 0, st, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  jl::jl_decode_combine_kernel<D><<<dim3(prm.Hq, B), jl::kCombineThreads, 0, st>>>(prm);
-  e = cudaGetLastError();
+  e = launch_pdl(jl::jl_decode_combine_kernel<D>, dim3(prm.Hq, B), dim3(jl::kCombineThreads), 0, st, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return ok();
 }
 
 template <int D, bool PLAIN>
 jl_status dispatch_group(const jl::DecodeParams& prm, int B, cudaStream_t st) {
-  if (decode_uses_tc(D, prm.Hq, prm.Hkv)) {
-    switch (prm.group) {
-      case 1: return launch_decode_tc<1, PLAIN>(prm, B, st);
-      case 2: return launch_decode_tc<2, PLAIN>(prm, B, st);
-      case 4: return launch_decode_tc<4, PLAIN>(prm, B, st);
-      case 8: return launch_decode_tc<8, PLAIN>(prm, B, st);
-      case 16: return launch_decode_tc<16, PLAIN>(prm, B, st);
-      default: break;
-    }
-  }
-  switch (prm.group) {
-    case 1: return launch_decode<D, 1, PLAIN>(prm, B, st);
-    case 2: return launch_decode<D, 2, PLAIN>(prm, B, st);
-    case 4: return launch_decode<D, 4, PLAIN>(prm, B, st);
-    case 8: return launch_decode<D, 8, PLAIN>(prm, B, st);
-    default: return fail(JL_ERR_UNSUPPORTED, "decode supports Hq/Hkv in {1, 2, 4, 8, 16} (got %d)", prm.group);
+  const int g = prm.group;
+  if (g < 1 || g > kMaxDecodeGroup)
+    return fail(JL_ERR_UNSUPPORTED, "decode supports 1 to %d query heads per KV head (got %d)", kMaxDecodeGroup, g);
+  if constexpr (D == 128) {  // tensor cores
+    if (g <= 1) return launch_decode_tc<1, PLAIN>(prm, B, st);
+    if (g <= 2) return launch_decode_tc<2, PLAIN>(prm, B, st);
+    if (g <= 4) return launch_decode_tc<4, PLAIN>(prm, B, st);
+    if (g <= 8) return launch_decode_tc<8, PLAIN>(prm, B, st);
+    return launch_decode_tc<16, PLAIN>(prm, B, st);
+  } else {  // head_dim 64: CUDA cores
+    if (g <= 1) return launch_decode<D, 1, PLAIN>(prm, B, st);
+    if (g <= 2) return launch_decode<D, 2, PLAIN>(prm, B, st);
+    if (g <= 4) return launch_decode<D, 4, PLAIN>(prm, B, st);
+    if (g <= 8) return launch_decode<D, 8, PLAIN>(prm, B, st);
+    return launch_decode<D, 16, PLAIN>(prm, B, st);
   }
 }
 
@@ -426,6 +469,14 @@ int64_t jl_group_size(int64_t L, int64_t w_pretrained) {
   return g < 1 ? 1 : g;
 }
 
+int jl_debug_bounds_enabled(void) {
+#ifdef JL_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 jl_status jl_sync_status(jl_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
@@ -439,9 +490,23 @@ jl_status jl_sync_status(jl_stream_t stream) {
     if (word & jl::kDevErrTimeout) return fail(JL_ERR_TIMEOUT, "a bounded in-kernel wait ran out");
     if (word & jl::kDevErrBounds)
       return fail(JL_ERR_INVALID, "a cache writer met a position outside the cache or the RoPE tables");
+    if (word & jl::kDevErrIndex)
+      return fail(JL_ERR_INVALID, "a debug-bounds check failed: a kernel derived an index outside its buffer");
   }
   return ok();
 }
+
+#ifdef JL_TRACE
+// Copies the timeline of the traced CTA (a build with -DJL_TRACE only).
+jl_status jl_debug_trace(long long* host, int n) {
+  const cudaError_t e = cudaMemcpyFromSymbol(host, jl::g_trace, sizeof(long long) * (n < 4096 ? n : 4096));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "trace copy");
+}
+jl_status jl_debug_trace_decode(long long* host, int n) {
+  const cudaError_t e = cudaMemcpyFromSymbol(host, jl::g_trace_dec, sizeof(long long) * (n < 1024 ? n : 1024));
+  return e == cudaSuccess ? ok() : cuda_fail(e, "trace copy");
+}
+#endif
 
 jl_status jl_selftest_wait_timeout(int64_t limit_cycles, jl_stream_t stream) {
   if (limit_cycles < 1000 || limit_cycles > 2000000000LL)
@@ -727,8 +792,8 @@ jl_status jl_plain_decode(const void* q, const void* k_cache, const void* v_cach
 // in jetlong.h).  The split-K partials live in one file-scope device array that
 // every GPU loading this library holds until the process exits.  Host code may
 // not pass the array's name to a kernel (on the host it is only a stand-in), so
-// the device address is looked up once per device with cudaGetSymbolAddress
-// while that device is current, then cached.
+// the device address is looked up with cudaGetSymbolAddress while that device is
+// current (see static_scratch_for).
 
 namespace {
 
@@ -739,17 +804,44 @@ constexpr int kMaxDevices = 128;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-jl_status static_scratch_for_current_device(void** addr) {
+// The scratch of the device the call runs on.  The kernels go to the caller's
+// stream, so that stream, the current device and the query buffer must all be on
+// one device: the array's address is only valid there.  Outside stream capture
+// the address is looked up again on every call (it changes if the device's
+// context was reset and the module reloaded); inside a capture the address from
+// the last uncaptured call on that device is used, so the first call on a device
+// must not be captured.
+jl_status static_scratch_for(cudaStream_t st, const void* q, void** addr) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(JL_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  int st_dev = -1;
+  e = cudaStreamGetDevice(st, &st_dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetDevice");
+  if (st_dev != dev)
+    return fail(JL_ERR_INVALID, "jl_bifocal_decode_noalloc: the stream belongs to device %d but device %d is current",
+                st_dev, dev);
+  cudaPointerAttributes pa{};
+  e = cudaPointerGetAttributes(&pa, q);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes(q)");
+  if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+    return fail(JL_ERR_INVALID, "jl_bifocal_decode_noalloc: q is not device memory");
+  if (pa.type == cudaMemoryTypeDevice && pa.device != dev)
+    return fail(JL_ERR_INVALID, "jl_bifocal_decode_noalloc: q lives on device %d but device %d is current", pa.device,
+                dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
     g_scratch_addr[dev] = p;
+  } else if (g_scratch_addr[dev] == nullptr) {
+    return fail(JL_ERR_INVALID,
+                "jl_bifocal_decode_noalloc: the first call on device %d must come before any stream capture", dev);
   }
   *addr = g_scratch_addr[dev];
   return JL_OK;
@@ -775,14 +867,18 @@ jl_status jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const vo
   if (B <= 0) return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim,
                                    w0, w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse,
                                    nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+  if (!q) return fail(JL_ERR_INVALID, "null pointer argument");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void* scratch = nullptr;
-  const jl_status s = static_scratch_for_current_device(&scratch);
+  const jl_status s = static_scratch_for(st, q, &scratch);
   if (s != JL_OK) return s;
   // Every partial the combine step reads is written earlier in the same call, so
-  // nothing in the scratch needs clearing between calls.
+  // nothing in the scratch needs clearing between calls.  If a split gives up (the
+  // device status word is set), the combine step writes NaN instead of blending
+  // stale partials.
   return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim, w0,
                        w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, scratch,
-                       kStaticScratchBytes, reinterpret_cast<cudaStream_t>(stream));
+                       kStaticScratchBytes, st);
 }
 
 }  // extern "C"

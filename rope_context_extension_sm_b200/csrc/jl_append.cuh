@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
 // rotate the query into q_out; rows Hq..Hq+Hkv-1 append key and value.
 template <int D>
 __global__ void __launch_bounds__(256) jl_decode_append_kernel(const AppendParams p) {
+  griddep_launch_dependents();  // the decode that follows may launch now; it waits for this grid to finish
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x & 31;
   const int per_b = p.Hq + p.Hkv;

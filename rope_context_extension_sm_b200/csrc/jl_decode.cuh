@@ -79,9 +79,13 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
   __shared__ float red_o[4][GROUP][D];
 
   const int hk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int ng = p.group;  // query heads of this KV head; GROUP is the capacity (rows >= ng stay zero)
+  griddep_wait();              // inputs may come from the previous kernel (see jl_device.cuh)
+  griddep_launch_dependents();
   const int L = p.seqlens[b];
   const int c0 = split * p.chunk;
   if (c0 >= L) return;
+  if (status_failed()) return;
   const int c1 = min(c0 + p.chunk, L);
   const int i = L - 1;
   int G = 1, jb = -1;  // remote keys are j <= jb
@@ -90,6 +94,10 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
     if (G > 1) jb = i - p.w0;
   }
   const int n0 = c0 - c0 / G;  // correction index j - f(j) of the chunk's first key
+  // the cache holds the length; the query's and the chunk's correction rows are in the table
+  // (a key's row n0 + t is formed by angle addition from rows n0 and t, checked per key)
+  JL_CHECK(L <= p.cache_stride && L <= p.n_split * p.chunk && (c1 - 1) - (c1 - 1) / G < p.n_tab_rows &&
+           (i - i / G) < p.n_tab_rows && hk * ng + ng <= p.Hq);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kg = lane >> 4, r = lane & 15;
@@ -128,10 +136,15 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
     float qr[GROUP][2 * H];
 #pragma unroll
     for (int g = 0; g < GROUP; ++g) {
-      const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * GROUP + g) * D;
       float lo[H], hi[H];
-      load_half_bf16<D>(qp + cl, lo);
-      load_half_bf16<D>(qp + HALFD + cl, hi);
+      if (g < ng) {
+        const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * ng + g) * D;
+        load_half_bf16<D>(qp + cl, lo);
+        load_half_bf16<D>(qp + HALFD + cl, hi);
+      } else {
+#pragma unroll
+        for (int e = 0; e < H; ++e) lo[e] = hi[e] = 0.f;
+      }
       if (remote) {  // R(f(i) - i) = R(-nq)
         const int64_t nq = i - i / G;
 #pragma unroll
@@ -162,6 +175,7 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
       load_half_bf16<D>(vp + HALFD + cl, vhi);
       if (remote) {  // R(f(j) - j) = R(-n_j), n_j = n0 + t, t < chunk
         const int t = (jj - jj / G) - n0;
+        JL_CHECK(t >= 0 && t < p.n_tab_rows);
         float cb[H], sb[H];
         load_f32<H>(p.cos_tab + static_cast<int64_t>(t) * HALFD + cl, cb);
         load_f32<H>(p.sin_tab + static_cast<int64_t>(t) * HALFD + cl, sb);
@@ -239,8 +253,8 @@ __global__ void __launch_bounds__(kDecodeThreads) jl_decode_split_kernel(const D
   }
   __syncthreads();
   // merge the four warps: thread handles (g, c) pairs
-  float* ws = p.ws + ((static_cast<int64_t>(b) * p.n_split + split) * p.Hq + hk * GROUP) * (D + 2);
-  for (int idx = threadIdx.x; idx < GROUP * D; idx += kDecodeThreads) {
+  float* ws = p.ws + ((static_cast<int64_t>(b) * p.n_split + split) * p.Hq + hk * ng) * (D + 2);
+  for (int idx = threadIdx.x; idx < ng * D; idx += kDecodeThreads) {
     const int g = idx / D, c = idx % D;
     float mx = -INFINITY;
 #pragma unroll
@@ -273,8 +287,17 @@ __global__ void __launch_bounds__(kCombineThreads) jl_decode_combine_kernel(cons
   constexpr int NW = kCombineThreads / 32;
   const int qh = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();  // launched while the split kernel runs: its partials are complete from here on
+  if (status_failed()) {  // a split gave up: its partials are stale, so the output is marked undefined
+    for (int c = threadIdx.x; c < D; c += kCombineThreads) {
+      p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(__int_as_float(0x7fc00000));
+      if (c == 0 && p.lse != nullptr) p.lse[static_cast<int64_t>(b) * p.Hq + qh] = __int_as_float(0x7fc00000);
+    }
+    return;
+  }
   const int L = p.seqlens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
+  JL_CHECK(L >= 1 && ns <= p.n_split);
   const float* base = p.ws + (static_cast<int64_t>(b) * p.n_split * p.Hq + qh) * (D + 2);
   const int64_t sstride = static_cast<int64_t>(p.Hq) * (D + 2);
   __shared__ float sm_red[NW], sm_l[NW];

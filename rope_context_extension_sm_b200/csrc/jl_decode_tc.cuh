@@ -1,5 +1,7 @@
 // jl_decode_tc.cuh -- split-K bifocal decode on sm_100a with the keys on the
-// tensor-core M dimension (head_dim 128, up to 16 query heads per KV head).
+// tensor-core M dimension (head_dim 128, up to 16 query heads per KV head; the
+// template GROUP is a capacity of 1, 2, 4, 8 or 16 heads and the runtime group
+// p.group <= GROUP picks the rows that hold real queries).
 //
 // Method: "Jet-Long: Efficient Long-Context Extension with Dynamic Bifocal
 // RoPE", Methodology section 2, on-the-fly correction rotation.  The cache holds
@@ -30,6 +32,21 @@
 #include "jl_device.cuh"
 
 namespace jl {
+
+// Optional timeline of one CTA (built only with -DJL_TRACE, for measurements):
+// SM clock stamps of the roles' events on the first 64 tiles of CTA (0, 1, 0).
+#ifdef JL_TRACE
+__device__ long long g_trace_dec[64 * 16];
+#define JL_DTRACE_AT(n, slot)                                                                           \
+  do {                                                                                                  \
+    if (blockIdx.x == 0 && blockIdx.y == 1 && blockIdx.z == 0 && (n) < 64 && (threadIdx.x & 31) == 0) \
+      g_trace_dec[(n) * 16 + (slot)] = clock64();                                                       \
+  } while (0)
+#else
+#define JL_DTRACE_AT(n, slot) \
+  do {                        \
+  } while (0)
+#endif
 
 constexpr int kDecTile = 128;    // keys per tile
 constexpr int kDecStages = 3;    // K/V pipeline depth
@@ -125,12 +142,28 @@ __device__ __forceinline__ void correct_slice(uint8_t* slice, int j0, int G, int
       }
     }
   } else {
+    // Any G: bit r of adv says whether n steps after row r (it does unless
+    // (j0 + r + 1) % G == 0), computed once per slice so the row loop carries no
+    // counter; the partial-slice test is hoisted out of the loop like above.
+    uint32_t adv = 0;
     int cnt = j0 % G;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
-      if (full || r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
       cnt = (cnt + 1 == G) ? 0 : cnt + 1;
-      step_factor(fc, fs, st_c, st_s, cnt != 0);
+      adv |= (cnt != 0 ? 1u : 0u) << r;
+    }
+    if (full) {
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        rotate_row_neg(slice, r, fc, fs, lane);
+        step_factor(fc, fs, st_c, st_s, (adv >> r) & 1u);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        if (r <= last_remote) rotate_row_neg(slice, r, fc, fs, lane);
+        step_factor(fc, fs, st_c, st_s, (adv >> r) & 1u);
+      }
     }
   }
 }
@@ -153,6 +186,9 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
   static_assert(GROUP <= kDecHeads, "up to 16 query heads per KV head");
 
   const int hk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int ng = p.group;  // query heads of this KV head (<= GROUP; the rest of the capacity is zero rows)
+  griddep_wait();              // the query, the cache rows and the lengths may come from the previous kernel
+  griddep_launch_dependents();  // the combine step may be scheduled now; it waits for this grid to finish
   const int L = p.seqlens[b];
   const int c0 = split * p.chunk;
   if (c0 >= L) return;
@@ -166,6 +202,8 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     if (G > 1) jb = i - p.w0;
   }
   const int64_t row0 = static_cast<int64_t>(b) * p.cache_stride;  // token row of this entry's first key
+  // the grid covers the length; the query's correction row is in the table
+  JL_CHECK(L <= p.n_split * p.chunk && i < p.n_tab_rows && (i - i / G) < p.n_tab_rows && hk * ng + ng <= p.Hq);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -222,7 +260,14 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
                              ? p.block_table[static_cast<int64_t>(b) * p.max_pages + kpos / p.page_size] * p.page_size +
                                    kpos % p.page_size
                              : static_cast<int>(row0) + kpos;
+        // contiguous: the tile's keys lie in entry b; paged: its page is inside the pool
+        JL_CHECK(kpos < L && (p.block_table != nullptr
+                                  ? (kpos / p.page_size < p.max_pages && key0 >= 0 &&
+                                     key0 + kDecTile <= p.cache_stride)
+                                  : L <= p.cache_stride));
+        JL_DTRACE_AT(n, 0);
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
+        JL_DTRACE_AT(n, 1);
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         tma_load_3d(sK + s * Lay::kTile, &tm_k, &bars->k_full[s], 0, hk, key0);
         tma_load_3d(sK + s * Lay::kTile + 16384, &tm_k, &bars->k_full[s], 64, hk, key0);
@@ -279,6 +324,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
           if (!(ok = mbar_wait(&bars->k_ready[s1], ((n + 1) / kDecStages) & 1, abort))) break;
           tc_fence_after();
           issue_s(n + 1);
+          JL_DTRACE_AT(n + 1, 5);
           umma_commit(&bars->s_full[(n + 1) & 1]);
           umma_commit(&bars->k_empty[s1]);
         }
@@ -286,6 +332,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
         tc_fence_after();
         const int s = n % kDecStages;
         if (!(ok = mbar_wait(&bars->v_full[s], (n / kDecStages) & 1, abort))) break;
+        JL_DTRACE_AT(n, 4);
         issue_pv(n);
         umma_commit(&bars->pv_done);
         umma_commit(&bars->v_empty[s]);
@@ -305,9 +352,13 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     auto anchor = [&](int n, float (&c)[2], float (&s)[2]) {
       const int j = c0 + n * kDecTile + Lay::kRotRows * rw;
       int64_t row = j - j / G;  // correction index n_j = j - f(j)
+      {
+        const int last = min(j + Lay::kRotRows - 1, c1 - 1);  // rows of the valid keys of this slice
+        JL_CHECK(j > last || last - last / G < p.n_tab_rows);
+      }
       row = row > p.n_tab_rows - 1 ? p.n_tab_rows - 1 : row;
-      const float2 cc = __ldg(reinterpret_cast<const float2*>(p.cos_tab + row * 64 + 2 * lane));
-      const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + row * 64 + 2 * lane));
+      const float2 cc = ldg_now_f2(p.cos_tab + row * 64 + 2 * lane);  // a tile ahead: issued here
+      const float2 ss = ldg_now_f2(p.sin_tab + row * 64 + 2 * lane);
       c[0] = cc.x; c[1] = cc.y; s[0] = ss.x; s[1] = ss.y;
     };
     float nc[2], ns[2];
@@ -317,6 +368,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       if (n + 1 < n_tiles) anchor(n + 1, nc, ns);
       const int s = n % kDecStages;
       if (!mbar_wait(&bars->k_full[s], (n / kDecStages) & 1, abort)) break;
+      if (rw == 0) JL_DTRACE_AT(n, 2);
       const int j0 = c0 + n * kDecTile + Lay::kRotRows * rw;  // key of this warp's first row
       const int last_remote = min(jb, c1 - 1) - j0;             // rows r <= last_remote are remote
       if (last_remote >= 0) {
@@ -332,6 +384,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);
+      if (rw == 0) JL_DTRACE_AT(n, 3);
     }
   } else {
     // ------------------------------------------------------------- softmax
@@ -346,8 +399,8 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
         const int row = e >> 6, c = e & 63;
         const int g = row & 15;
         float lo = 0.f, hi = 0.f;
-        if (g < GROUP) {
-          const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * GROUP + g) * 128;
+        if (g < ng) {
+          const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * ng + g) * 128;
           lo = __bfloat162float(qp[c]);
           hi = __bfloat162float(qp[c + 64]);
           if (row < 16 && G > 1 && !PLAIN) {
@@ -376,6 +429,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     bool ok = true;
     for (int n = 0; n < n_tiles && ok; ++n) {
       if (!(ok = mbar_wait(&bars->s_full[n & 1], (n >> 1) & 1, abort))) break;
+      if (wq == 0) JL_DTRACE_AT(n, 6);
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld32(t_lane + (n & 1) * 32, sr);
@@ -397,6 +451,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       }
       mbar_arrive(&bars->red_full[n & 1]);
       if (!(ok = mbar_wait(&bars->red_full[n & 1], (n >> 1) & 1, abort))) break;
+      if (wq == 0) JL_DTRACE_AT(n, 7);
       float alpha[GROUP];
       bool any_resc = false;
 #pragma unroll
@@ -410,6 +465,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       }
       // PV(n-1) must be complete before P buffer (n & 1) is rewritten and before O is rescaled
       if (n > 0 && !(ok = mbar_wait(&bars->pv_done, (n - 1) & 1, abort))) break;
+      if (wq == 0) JL_DTRACE_AT(n, 8);
       tc_fence_after();
       uint8_t* pb = sP + (n & 1) * (kDecHeads * 256);
 #pragma unroll
@@ -429,6 +485,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->p_ready[n & 1]);
+      if (wq == 0) JL_DTRACE_AT(n, 9);
     }
     // epilogue: row sums across the 128 threads, then the partial per query head
     if (ok && mbar_wait(&bars->pv_done, (n_tiles - 1) & 1, abort)) {
@@ -445,9 +502,10 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       if (mbar_wait(&bars->red_end, 0, abort)) {
       uint32_t o[32];
       tmem_ld32(t_lane + 64, o);  // thread = channel tid
-      float* ws = p.ws + ((static_cast<int64_t>(b) * p.n_split + split) * p.Hq + hk * GROUP) * (128 + 2);
+      float* ws = p.ws + ((static_cast<int64_t>(b) * p.n_split + split) * p.Hq + hk * ng) * (128 + 2);
 #pragma unroll
       for (int g = 0; g < GROUP; ++g) {
+        if (g >= ng) break;
         float* dst = ws + static_cast<int64_t>(g) * (128 + 2);
         dst[2 + tid] = __uint_as_float(o[g]);
         if (tid == 0) {

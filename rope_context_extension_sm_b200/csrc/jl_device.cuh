@@ -14,8 +14,25 @@ namespace jl {
 
 // Device status word bits (read and cleared by jl_sync_status).
 constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrIndex = 4u;  // a debug-bounds check failed (see JL_CHECK)
 // Defined here: the library is a single translation unit (csrc/jetlong.cu).
 __device__ unsigned int g_status = 0;
+
+// Debug-bounds build (-DJL_DEBUG_BOUNDS): device-side checks of the indices the
+// kernels derive on the device (table rows, TMA tile coordinates, cache and page
+// positions, workspace slots).  A failed check records kDevErrIndex in the status
+// word and execution continues (no trap); jl_sync_status reports it.  In the
+// normal build the checks compile to nothing.
+#ifdef JL_DEBUG_BOUNDS
+#define JL_CHECK(cond)                                                      \
+  do {                                                                      \
+    if (!(cond)) atomicOr(&::jl::g_status, ::jl::kDevErrIndex);             \
+  } while (0)
+#else
+#define JL_CHECK(cond) \
+  do {                 \
+  } while (0)
+#endif
 
 // A bounded wait gives up after this many SM clock cycles (~0.2-0.3 s); every
 // legitimate wait in these kernels is microseconds long.
@@ -45,6 +62,22 @@ __device__ __forceinline__ void fence_mbar_init() {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Arrive that cannot be issued before `dep` is computed: the value is an input of
+// the instruction, so every operation feeding it (e.g. a row sum over the
+// exponentials) completes first.
+__device__ __forceinline__ void mbar_arrive_after(uint64_t* bar, float dep) {
+  asm volatile("{\n .reg .f32 d;\n mov.b32 d, %1;\n mbarrier.arrive.shared::cta.b64 _, [%0];\n}\n" ::"r"(smem_u32(bar)),
+               "f"(dep)
+               : "memory");
+}
+
+// Returns x through an opaque move, so work that uses the result is not started
+// before the preceding (volatile) instructions, e.g. a barrier wait.
+__device__ __forceinline__ float order_after(float x) {
+  asm volatile("mov.b32 %0, %0;" : "+f"(x)::"memory");
+  return x;
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -272,6 +305,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 
 // ------------------------------------------------------------------- misc --
 
+// Read-only global loads issued exactly where they are written: volatile asm is
+// not moved past the other volatile asm around it (the barrier waits), so a
+// prefetch a tile ahead stays a tile ahead instead of being sunk to its first use.
+__device__ __forceinline__ float2 ldg_now_f2(const float* p) {
+  float2 r;
+  asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(r.x), "=f"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ float ldg_now_f(const float* p) {
+  float r;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r) : "l"(p));
+  return r;
+}
+
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: two lanes of work per instruction).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -320,6 +367,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Two finite floats to a bf16 pair on the integer pipe: half a bf16 ulp is added
+// to each bit pattern (rounding the magnitude to nearest, ties away from zero)
+// and the two upper halves are byte-permuted together.  Differs from the
+// round-to-nearest-even conversion only on exact ties.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
+#ifndef JL_IPACK
+#define JL_IPACK 0  // 1: P packed on the integer pipe; 2: the rotations' outputs too
+#endif
+
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 // Register reallocation between warpgroups (all four warps of a warpgroup
@@ -333,6 +392,17 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Programmatic dependent launch (sm_90 and later).  A kernel launched with the
+// programmatic stream-serialization attribute may start while the previous
+// kernel of its stream is still running; griddep_wait() returns once that kernel
+// has completed and its writes are visible, so it must come before every read of
+// data an earlier kernel produced (without the attribute it returns at once).
+// griddep_launch_dependents() lets the next such kernel start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // One lane of the (converged) warp is elected; the others get false.

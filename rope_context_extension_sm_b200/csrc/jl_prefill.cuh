@@ -24,17 +24,18 @@
 //   warp 0      TMA producer (Q, K, V tiles; 128B-swizzled boxes)
 //   warp 1      TMEM allocator + tcgen05.mma issuer (warp-uniform loop, one
 //               elected lane issues)
-//   warps 2, 3  in-place RoPE rotation of the Q and K tiles in shared memory
-//   and two     (base rows R(x) or remote rows R(f(x))); each owns 32 rows and
-//   more        steps its cos/sin factors along the rows by complex
-//               multiplication with e^{i theta_c}, anchored once per tile on a
-//               table row prefetched a tile ahead (no table load per row)
+//   warps 2, 3  idle (the control warpgroup is complete for the register split)
 //   warps 4..   one warpgroup per query head: the whole 128-column score row of
 //               each thread read from TMEM once per tile, softmax in registers,
 //               P written back to TMEM (bf16), O rescale, epilogue
-//   last two    idle (every warpgroup is complete for the register split)
+//   last four   in-place RoPE rotation of the Q and K tiles in shared memory
+//               (base rows R(x) or remote rows R(f(x))); each owns 32 rows and
+//               steps its cos/sin factors along the rows by complex
+//               multiplication with e^{i theta_c}, anchored once per tile on a
+//               table row prefetched a tile ahead (no table load per row)
 // Registers: launched at 65536 / threads per thread; setmaxnreg moves them from
-// the producer / MMA / rotation / idle warpgroups (56) to the softmax ones (200).
+// the control warpgroup (48) and the rotation warpgroup (64) to the softmax
+// ones (200).
 // TMEM columns: S_t at 128 t, O_t at 128 NQT + D t; P_t aliases S_t.
 // With NQT = 2 the MMA issue order S0(n), PV1(n-1), S1(n), PV0(n) lets one
 // head's softmax overlap the other head's tensor-core work.
@@ -47,6 +48,21 @@ namespace jl {
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr int kStages = 2;
+
+// Optional timeline of one CTA (built only with -DJL_TRACE, for measurements):
+// SM clock stamps of the roles' events on visits 100 .. 163 of CTA 0.
+#ifdef JL_TRACE
+__device__ long long g_trace[64 * 64];
+#define JL_TRACE_AT(n, slot)                                                     \
+  do {                                                                           \
+    if (blockIdx.x == 0 && (n) >= 100 && (n) < 164 && (threadIdx.x & 31) == 0) \
+      g_trace[((n) - 100) * 64 + (slot)] = clock64();                            \
+  } while (0)
+#else
+#define JL_TRACE_AT(n, slot) \
+  do {                       \
+  } while (0)
+#endif
 
 struct PrefillParams {
   const int32_t* cu_seqlens;
@@ -95,25 +111,26 @@ struct PrefillLayout {
   static constexpr int kColsUsed = NQT * 128 + NQT * D;
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256u : 512u;
   static constexpr int kRotWarps = 4;
-  // warps: 0 producer, 1 MMA, 2-3 rotation, 4 .. kR0-1 softmax (one warpgroup
-  // per query head), kR0 and kR0+1 rotation, kR0+2 and kR0+3 idle (every
-  // warpgroup is complete, as the register split requires).
+  // Warpgroups: 0 = control (warp 0 TMA producer, warp 1 MMA issuer, warps 2-3
+  // idle), 1 .. NQT = softmax (one per query head), NQT + 1 = rotation (warps
+  // kR0 .. kR0 + 3).  Every warpgroup is complete, as the register split requires.
   static constexpr int kR0 = 4 + 4 * NQT;
   static constexpr int kWarps = kR0 + 4;
   static constexpr int kThreads = 32 * kWarps;
-  // The softmax warpgroups hold a whole 128-column score row in registers.  The
-  // block is launched at kRegsLaunch registers per thread; the producer / MMA /
-  // rotation warpgroups give theirs down to kRegsOther and the softmax
-  // warpgroups take kRegsSoftmax.  Two heads: 128 x (2 x 200 + 2 x 56) = 512 x 128.
+  // The softmax warpgroups hold a whole 128-column score row in registers and the
+  // rotation warpgroup keeps eight rows of a tile in flight.  The block is
+  // launched at kRegsLaunch registers per thread; the control warpgroup gives its
+  // registers down to kRegsCtl and the rotation warpgroup to kRegsRot, the
+  // softmax warpgroups take kRegsSoftmax.  Two heads: 128 x (48 + 2 x 200 + 64) =
+  // 512 x 128, the whole register file.
   static constexpr bool kSplitRegs = true;
   static constexpr uint32_t kRegsLaunch = (65536 / kThreads) & ~7u;
-  static constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 56;
-  static constexpr uint32_t kRegsNeeded = 128 * (NQT * kRegsSoftmax + (kWarps / 4 - NQT) * kRegsOther);
+  static constexpr uint32_t kRegsSoftmax = 200, kRegsCtl = 48, kRegsRot = 64;
+  static constexpr uint32_t kRegsNeeded = 128 * (NQT * kRegsSoftmax + kRegsCtl + kRegsRot);
   static_assert(kRegsNeeded <= kThreads * kRegsLaunch, "register split exceeds the launch allocation");
+  static_assert(kRegsRot <= kRegsLaunch && kRegsCtl <= kRegsLaunch, "a decrease must not exceed the launch count");
   __device__ static bool softmax_warp(int warp) { return warp >= 4 && warp < kR0; }
-  __device__ static int rot_index(int warp) {
-    return (warp == 2 || warp == 3) ? warp - 2 : ((warp == kR0 || warp == kR0 + 1) ? warp - kR0 + 2 : -1);
-  }
+  __device__ static int rot_index(int warp) { return (warp >= kR0 && warp < kR0 + 4) ? warp - kR0 : -1; }
 };
 
 struct PrefillBars {
@@ -121,6 +138,7 @@ struct PrefillBars {
   uint64_t k_full[kStages], k_ready[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_ready[2], o_final[2];
+  uint64_t ex_done[2];  // head t's softmax warpgroup finished the exponentials of a tile
   uint64_t teardown;
   uint32_t tmem_base;
   int abort;
@@ -186,12 +204,12 @@ __device__ __forceinline__ void load_factor(RotFactor<D>& f, const PrefillParams
   const int64_t max_row = (rem ? p.n_rem_rows : p.n_tab_rows) - 1;
   row = row > max_row ? max_row : row;  // only rows past every sequence end are clamped
   if constexpr (D == 128) {
-    const float2 cc = __ldg(reinterpret_cast<const float2*>(ct + row * 64 + 2 * lane));
-    const float2 ss = __ldg(reinterpret_cast<const float2*>(st + row * 64 + 2 * lane));
+    const float2 cc = ldg_now_f2(ct + row * 64 + 2 * lane);
+    const float2 ss = ldg_now_f2(st + row * 64 + 2 * lane);
     f.c[0] = cc.x; f.c[1] = cc.y; f.s[0] = ss.x; f.s[1] = ss.y;
   } else {
-    f.c[0] = __ldg(ct + row * 32 + lane);
-    f.s[0] = __ldg(st + row * 32 + lane);
+    f.c[0] = ldg_now_f(ct + row * 32 + lane);
+    f.s[0] = ldg_now_f(st + row * 32 + lane);
   }
 }
 
@@ -286,9 +304,79 @@ __device__ __forceinline__ void rotate_slice(uint8_t* tile, int rw, int base, in
   }
 }
 
+#ifdef JL_ROT_B8
+// head_dim 128: rows [32 rw, 32 rw + 32) in four batches of eight rows -- every
+// load of a batch first, then the arithmetic, then the stores -- so eight rows'
+// shared-memory loads are in flight together instead of one row at a time.  Row
+// r = 8 k + e of the slice has r & 7 == e, so its swizzled offset is known at
+// compile time up to the lane.  f steps by st every g rows (GS > 0: g == GS).
+template <int GS>
+__device__ __forceinline__ void rotate_slice_b8(uint8_t* tile, int rw, int base, int g, RotFactor<128> f,
+                                                const RotFactor<128>& st, int lane) {
+  uint8_t* slice = tile + 32 * rw * 128;
+  int cnt = GS > 0 ? 0 : (base + 32 * rw) % g;
+#pragma unroll 1
+  for (int r0 = 0; r0 < 32; r0 += 8) {
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int off = (r0 + e) * 128 + (((lane >> 2) ^ e) << 4) + ((lane & 3) << 2);
+      lo[e] = *reinterpret_cast<const uint32_t*>(slice + off);
+      hi[e] = *reinterpret_cast<const uint32_t*>(slice + 16384 + off);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo[e]));
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[e]));
+      const uint64_t c2 = f2_pack(f.c[0], f.c[1]);
+      const uint64_t s2 = f2_pack(f.s[0], f.s[1]), ns2 = f2_pack(-f.s[0], -f.s[1]);
+      const uint64_t a2 = f2_pack(a.x, a.y), b2 = f2_pack(b.x, b.y);
+      float2 ya, yb;
+      f2_unpack(f2_fma(b2, ns2, f2_mul(a2, c2)), ya.x, ya.y);
+      f2_unpack(f2_fma(a2, s2, f2_mul(b2, c2)), yb.x, yb.y);
+      lo[e] = JL_IPACK >= 2 ? pack_bf16x2_alu(ya.x, ya.y) : pack_bf16x2(ya.x, ya.y);
+      hi[e] = JL_IPACK >= 2 ? pack_bf16x2_alu(yb.x, yb.y) : pack_bf16x2(yb.x, yb.y);
+      if constexpr (GS > 0) {
+        if ((e + 1) % GS == 0) advance<128>(f, st);
+      } else {
+        cnt = (cnt + 1 == g) ? 0 : cnt + 1;
+        RotFactor<128> nf = f;
+        advance<128>(nf, st);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          f.c[q] = cnt == 0 ? nf.c[q] : f.c[q];
+          f.s[q] = cnt == 0 ? nf.s[q] : f.s[q];
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int off = (r0 + e) * 128 + (((lane >> 2) ^ e) << 4) + ((lane & 3) << 2);
+      *reinterpret_cast<uint32_t*>(slice + off) = lo[e];
+      *reinterpret_cast<uint32_t*>(slice + 16384 + off) = hi[e];
+    }
+  }
+}
+#endif
+
 template <int D>
 __device__ __forceinline__ void rotate_slice_any(uint8_t* tile, int rw, int base, int g, const RotFactor<D>& f,
                                                  const RotFactor<D>& st, int lane) {
+#ifdef JL_ROT_B8
+  if constexpr (D == 128) {
+    if ((base & 31) != 0) {
+      rotate_slice_b8<0>(tile, rw, base, g, f, st, lane);
+      return;
+    }
+    switch (g) {
+      case 1: rotate_slice_b8<1>(tile, rw, base, g, f, st, lane); break;
+      case 2: rotate_slice_b8<2>(tile, rw, base, g, f, st, lane); break;
+      case 4: rotate_slice_b8<4>(tile, rw, base, g, f, st, lane); break;
+      default: rotate_slice_b8<0>(tile, rw, base, g, f, st, lane); break;
+    }
+    return;
+  }
+#endif
   if ((base & 31) != 0) {  // a chunk's query block need not start on a multiple of 32
     rotate_slice<D, 0>(tile, rw, base, g, f, st, lane);
     return;
@@ -349,12 +437,45 @@ __device__ __forceinline__ void write_cache_slice(const uint8_t* tile, int rw, c
     const int r = r0 + lane / kChunks;    // row within the slice
     const int row = 32 * rw + r;          // row within the tile
     if (row >= n_valid) continue;
+    JL_CHECK(pos0 + row < p.cache_out_stride && v_tok0 + row < p.total_tokens && b < p.batch);
     const uint4 kw = *reinterpret_cast<const uint4*>(tile + box * 16384 + row * 128 + ((j ^ (row & 7)) << 4));
     const int64_t dst = ((static_cast<int64_t>(b) * p.cache_out_stride + pos0 + row) * p.Hkv + hkv) * D + c * 8;
     const int64_t src = ((v_tok0 + row) * p.Hkv + hkv) * D + c * 8;
     *reinterpret_cast<uint4*>(p.k_cache_out + dst) = kw;
     *reinterpret_cast<uint4*>(p.v_cache_out + dst) = *reinterpret_cast<const uint4*>(p.v_raw + src);
   }
+}
+
+// Every JL_POLY_EVERY-th pair of exponentials of a score row is computed on the
+// FMA pipe instead of the MUFU unit, which both heads' softmax share (0: none).
+#ifndef JL_POLY_EVERY
+#define JL_POLY_EVERY 0
+#endif
+
+// 2^x for a pair of values on the FMA and integer pipes.  Range reduction: the
+// nearest integer n of x comes from adding 1.5 * 2^23 (its low bits then hold n),
+// f = x - n lies in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted for
+// minimum relative error on that interval (at most 7.5e-5, far below the bf16
+// rounding P gets); 2^n is added into the exponent field.  x is clamped to
+// >= -125 so the result stays a normal number.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float& y0, float& y1) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t shift = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(xc, shift);
+  const uint64_t fr = f2_sub(xc, f2_sub(t, shift));
+  uint64_t pl = f2_fma(fr, f2_pack(0.05517160892486572f, 0.05517160892486572f),
+                       f2_pack(0.2426111102104187f, 0.2426111102104187f));
+  pl = f2_fma(pl, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  pl = f2_fma(pl, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(pl, q0, q1);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // p = 2^(s * sl2 - m) over NC score columns (zero outside [keep_lo + 1,
@@ -369,17 +490,22 @@ __device__ __forceinline__ void softmax_chunk(const uint32_t (&sr)[NC], uint32_t
   for (int e = 0; e < NC / 2; ++e) {
     // (s0, s1) * scale - m in one packed FMA, two ex2, one packed add into the row sums
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), scale2, negm2);
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    float p0 = ex2_approx(x0);
-    float p1 = ex2_approx(x1);
+    float p0, p1;
+    if (JL_POLY_EVERY > 0 && e % (JL_POLY_EVERY > 0 ? JL_POLY_EVERY : 1) == JL_POLY_EVERY - 1) {
+      exp2_poly_x2(x, p0, p1);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
     if constexpr (MASK) {
       const int col = col0 + 2 * e;
       p0 = (col > keep_lo && col <= keep_hi) ? p0 : 0.f;
       p1 = (col + 1 > keep_lo && col + 1 <= keep_hi) ? p1 : 0.f;
     }
     acc = f2_add(acc, f2_pack(p0, p1));
-    pk[e] = pack_bf16x2(p0, p1);
+    pk[e] = JL_IPACK >= 1 ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
   }
   f2_unpack(acc, lsum, lsum2);
 }
@@ -465,6 +591,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_ready[t], 128);
       mbar_init(&bars->o_final[t], 1);
+      mbar_init(&bars->ex_done[t], 128);
     }
     mbar_init(&bars->teardown, 1);
     bars->abort = 0;
@@ -480,8 +607,8 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   // Register split: each role's first instruction, executed by the whole warp
   // (every warp of a warpgroup takes the same share).
-  auto give_regs = [] {
-    if constexpr (Lay::kSplitRegs) setmaxnreg_dec<Lay::kRegsOther>();
+  auto give_regs = [] {  // control warpgroup
+    if constexpr (Lay::kSplitRegs) setmaxnreg_dec<Lay::kRegsCtl>();
   };
 
   if (warp == 0) {
@@ -493,6 +620,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       tma_prefetch_desc(&tm_v);
       int issued_q = 0;
       int issued[kStages] = {0};
+      JL_CHECK(q_tok0 >= 0 && q_tok0 < p.total_tokens && h0 + NQT <= p.Hq && hkv < p.Hkv);
       for (int n = 0; n < sc.n_virt && !*abort; ++n) {
         if (sc.phase_start(n)) {
           if (n > 0 && !mbar_wait(&bars->q_empty, 0, abort)) break;
@@ -506,6 +634,11 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         const int s = n % kStages;
         const uint32_t u = n / kStages;
         const int key0 = p.cached ? static_cast<int>(b * p.cache_stride) + sc.kt(n) * kBN : seq0 + sc.kt(n) * kBN;
+        // the tile's causal keys lie inside this sequence's keys (packed prompt or cache entry)
+        JL_CHECK(key0 >= 0 && sc.kt(n) * kBN < L &&
+                 key0 + min(kBN - 1, L - 1 - sc.kt(n) * kBN) <
+                     (p.cached ? static_cast<int64_t>(b) * p.cache_stride + (L < p.cache_stride ? L : p.cache_stride)
+                               : static_cast<int64_t>(seq0) + n_rows));
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         for (int bx = 0; bx < NBOX; ++bx)
@@ -565,7 +698,9 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       }
       const int s = n % kStages;
       const uint32_t u = n / kStages;
+      JL_TRACE_AT(n, 0);
       if (!(ok = warp_wait(&bars->k_ready[s], u & 1, abort))) break;
+      JL_TRACE_AT(n, 1);
       tc_fence_after();
       issue_s(0, s);
       commit(&bars->s_full[0]);
@@ -580,10 +715,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         }
         issue_s(1, s);
         commit(&bars->s_full[1]);
+        JL_TRACE_AT(n, 3);
       }
       commit(&bars->k_empty[s]);
       if (sc.phase_end(n)) commit(&bars->q_empty);
+      JL_TRACE_AT(n, 2);
       if (!(ok = warp_wait(&bars->p_ready[0], n & 1, abort))) break;
+      JL_TRACE_AT(n, 4);
       tc_fence_after();
       if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
       issue_pv(0, s, n > 0);
@@ -611,7 +749,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     mbar_wait_bounded(&bars->teardown, 0);
     __syncwarp();
   } else if (Lay::rot_index(warp) >= 0) {
-    give_regs();
+    if constexpr (Lay::kSplitRegs) setmaxnreg_dec<Lay::kRegsRot>();
     // ------------------------------------------------------------ rotation
     const int rw = Lay::rot_index(warp);
     RotFactor<D> step, step_rem;  // e^{i theta_c} (row 1 of the base table) and of the interpolated table
@@ -635,6 +773,11 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (sc.phase_start(n)) {
         RotFactor<D> fq;
         load_factor<D>(fq, p, slice_anchor_row(sc.q_lo, rw, g), lane, rem_tab);
+        {  // table rows of this slice's valid query rows
+          const int first = sc.q_lo + 32 * rw, last = min(first + 31, L - 1);
+          JL_CHECK(first > last || (last / g < (rem_tab ? p.n_rem_rows : p.n_tab_rows) &&
+                                    (g == 1 || interp || last / g < p.w_pre)));
+        }
         if (!mbar_wait(&bars->q_full, n == 0 ? 0 : 1, abort)) break;
         for (int t = 0; t < NQT; ++t) rotate_slice_any<D>(sQ + t * Lay::kTileBytes, rw, sc.q_lo, g, fq, stp, lane);
         fence_proxy_async_smem();
@@ -645,7 +788,18 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       if (n + 1 < sc.n_virt)  // prefetch a tile ahead
         load_factor<D>(fk_next, p, key_anchor(n + 1), lane, interp && sc.remote(n + 1));
       const int s = n % kStages;
+      {  // table rows of this slice's valid keys: base R(j), remote R(j / G) (< w_pretrained), or the
+         // cached keys' correction rows j - j / G
+        const int first = sc.kt(n) * kBN + 32 * rw, last = min(first + 31, L - 1);
+        if (p.cached)
+          JL_CHECK(first > last || g == 1 || last - last / G < p.n_tab_rows);
+        else
+          JL_CHECK(first > last || (last / g < (rem_tab ? p.n_rem_rows : p.n_tab_rows) &&
+                                    (g == 1 || interp || last / g < p.w_pre)));
+      }
+      JL_TRACE_AT(n, 5 + 3 * rw);
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
+      JL_TRACE_AT(n, 6 + 3 * rw);
       if (!p.cached) {
         rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, stp, lane);
         // The query block's own key tile, visited as local, now holds R(j) k_j: the first
@@ -665,6 +819,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->k_ready[s]);
+      JL_TRACE_AT(n, 7 + 3 * rw);
     }
   } else if (Lay::softmax_warp(warp)) {
     if constexpr (Lay::kSplitRegs) setmaxnreg_inc<Lay::kRegsSoftmax>();
@@ -682,6 +837,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     bool ok = true;
     for (int n = 0; n < sc.n_virt; ++n) {
       if (!(ok = mbar_wait(&bars->s_full[t], n & 1, abort))) break;
+      JL_TRACE_AT(n, 20 + 20 * t + 5 * wq);
       tc_fence_after();
       // The whole score row in registers: one TMEM round trip per tile.
       uint32_t sr[128];
@@ -712,14 +868,28 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       const bool resc = (m_run != -INFINITY) && (m_new > m_run + 8.f);
       const float alpha = resc ? ex2_approx(m_run - m_new) : 1.f;
       if (resc || m_run == -INFINITY) m_run = m_new;
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      JL_TRACE_AT(n, 21 + 20 * t + 5 * wq);
+      // The two heads take turns on the exponential unit: head 0's exponentials of
+      // tile n, then head 1's of tile n, then head 0's of tile n + 1, ...  Run at the
+      // same time they would share it and each take about twice as long, which
+      // lengthens both heads' S -> softmax -> PV chains; one at a time, each runs at
+      // the unit's full rate while the other loads and reduces its next scores.
+      if (NQT == 2 && (t == 1 || n > 0)) {
+        const uint32_t par = static_cast<uint32_t>(t == 1 ? n : n - 1) & 1u;
+        if (!(ok = mbar_wait(&bars->ex_done[1 - t], par, abort))) break;
+        m_use = order_after(m_use);
+      }
+      JL_TRACE_AT(n, 22 + 20 * t + 5 * wq);
       // P = 2^(s * scale_log2 - m) as bf16 pairs over S columns [0, 64).
       float lsum = 0.f, lsum2 = 0.f;
       uint32_t pk[64];
       if (msk) softmax_chunk<true, 128>(sr, pk, 0, sl2, -m_use, keep_lo, keep_hi, lsum, lsum2);
       else softmax_chunk<false, 128>(sr, pk, 0, sl2, -m_use, keep_lo, keep_hi, lsum, lsum2);
-      tmem_st64(t_s, pk);
       lsum += lsum2;
+      if (NQT == 2) mbar_arrive_after(&bars->ex_done[t], lsum);
+      JL_TRACE_AT(n, 23 + 20 * t + 5 * wq);
+      tmem_st64(t_s, pk);
       l_run = l_run * alpha + lsum;
       // O_t *= alpha for the rows whose max moved (PV_t(n-1) is complete: it was
       // issued before S_t(n), whose commit we waited on).
@@ -736,11 +906,13 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&bars->p_ready[t]);
+      JL_TRACE_AT(n, 24 + 20 * t + 5 * wq);
     }
     if (ok && mbar_wait(&bars->o_final[t], 0, abort)) {
       tc_fence_after();
       const int h = h0 + t;
       const bool valid = i <= sc.q_hi;
+      JL_CHECK(!valid || (static_cast<int64_t>(q_tok0) + row < p.total_tokens && h < p.Hq));
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const int64_t row_off = ((static_cast<int64_t>(q_tok0) + row) * p.Hq + h) * D;
 #pragma unroll
@@ -773,7 +945,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
     }
   }
 
-  if (warp >= Lay::kR0 + 2) give_regs();  // idle warps (two-head layout) still give their share
+  if (warp == 2 || warp == 3) give_regs();  // the control warpgroup's idle warps still give their share
 
   // ---- teardown: every role is done; TMEM is released by its allocator warp ----
   tc_fence_before();

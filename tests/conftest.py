@@ -11,3 +11,10 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def pytest_terminal_summary(terminalreporter):
+    import _headroom
+    if _headroom.RECORDS:
+        for line in _headroom.summary_lines(2e-2, 2e-3, 1e-2):
+            terminalreporter.write_line(line)

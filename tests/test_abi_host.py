@@ -84,7 +84,7 @@ def _call_decode(jlmod, **over):
 
 
 @pytest.mark.parametrize("over,status", [
-    (dict(d=80), 2), (dict(Hq=24, Hkv=8), 2), (dict(Hq=30), 1), (dict(stride=512), 1), (dict(n_tab=10), 1),
+    (dict(d=80), 2), (dict(Hq=34, Hkv=2), 2), (dict(Hq=30), 1), (dict(stride=512), 1), (dict(n_tab=10), 1),
     (dict(ws_bytes=10), 1), (dict(ws=None), 1), (dict(k=8), 1), (dict(max_seqlen=0), 1), (dict(w0=-3), 1),
 ])
 def test_decode_rejects_bad_arguments_without_launching(jlmod, over, status):

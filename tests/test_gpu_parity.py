@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 import torch
 
+import _headroom
 from oracle import oracle as O
 from rope_context_extension_sm_b200 import inputs as I
 
@@ -38,6 +39,7 @@ def _check(got_out, got_lse, ref_out, ref_lse, what):
     assert err.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e}"
     assert err.mean() <= OUT_MEAN, f"{what}: out mean-abs {err.mean():.3e}"
     assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
+    _headroom.record(what, err.max(), err.mean(), lerr.max())
     return err.max(), err.mean(), lerr.max()
 
 
@@ -258,6 +260,63 @@ def test_small_decode_steps(jl, L):
     _check(out[0], lse[0], ro, rl, f"plain decode L={L}")
 
 
+DECODE_GROUPS = [
+    # name, Hq, Hkv, head_dim: head_dim 64 runs the CUDA-core split kernel, 128 the tensor-core one;
+    # groups between the built capacities (1, 2, 4, 8, 16) run in the next capacity up
+    ("d64_g1", 2, 2, 64),
+    ("d64_g2", 4, 2, 64),
+    ("d64_g3", 6, 2, 64),
+    ("d64_g4", 8, 2, 64),
+    ("d64_g8", 8, 1, 64),
+    ("d64_g16", 16, 1, 64),
+    ("d128_g3", 6, 2, 128),
+    ("d128_g12", 12, 1, 128),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_GROUPS, ids=[c[0] for c in DECODE_GROUPS])
+@pytest.mark.parametrize("L", [1, 100, 101, 255, 256, 257])
+def test_decode_head_dims_and_groups(jl, case, L):
+    """Bifocal and plain decode against the oracle for every decode kernel and GQA shape:
+    w0 = 40, w_pretrained = 64, so these lengths give G = 1, 2, 2, 4, 4, 5."""
+    name, hq, hkv, d = case
+    cfg = I.DecodeConfig(name, (), hq, hkv, d, 40, 64, 1e4)
+    max_len = 300
+    k_cache, v = _decode_setup(cfg, max_len)
+    q_t = _query_tilde(cfg, I.decode_queries(cfg, 1)[0, 0], L)
+    cos, sin = _tables(jl, max_len, d, cfg.rope_base)
+    for plain in (False, True):
+        out, lse = _run_decode(jl, cfg, q_t[None], k_cache.cuda(), v.cuda(), [L], max_len, cos, sin, plain=plain)
+        ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L, plain=plain)
+        _check(out[0], lse[0], ro, rl, f"{name} {'plain' if plain else 'bifocal'} decode L={L}")
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (6, 2)])
+def test_decode_d64_batched_and_long(jl, hq, hkv):
+    """head_dim 64 (CUDA-core kernel): a batch whose entries each have their own G, with a cache
+    long enough that the split size grows past its minimum (20000 keys: 128-key chunks)."""
+    cfg = I.DecodeConfig("d64_batch", (), hq, hkv, 64, 100, 1024, 1e4)
+    max_len, lens = 20000, [20000, 1024, 1025, 7, 5000]
+    k_cache, v = _decode_setup(cfg, max_len, batch=len(lens))
+    qs = I.decode_queries(cfg, 1, batch=len(lens))[0]
+    q_t = torch.stack([_query_tilde(cfg, qs[b], lens[b]) for b in range(len(lens))])
+    cos, sin = _tables(jl, max_len, 64, cfg.rope_base)
+    out, lse = _run_decode(jl, cfg, q_t, k_cache.cuda(), v.cuda(), lens, max_len, cos, sin)
+    for b, L in enumerate(lens):
+        ro, rl = _decode_oracle(cfg, q_t[b], k_cache[b], v[b], L)
+        _check(out[b], lse[b], ro, rl, f"d64 batched decode b={b} L={L} G={O.group_size(L, 1024)}")
+
+
+def test_decode_refuses_more_than_16_heads_per_kv_head(jl):
+    cfg = I.DecodeConfig("g32", (), 32, 1, 128, 40, 64, 1e4)
+    k_cache, v = _decode_setup(cfg, 64)
+    cos, sin = _tables(jl, 64, 128, cfg.rope_base)
+    q = torch.zeros((1, 32, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(jl.JetLongError) as err:
+        _run_decode(jl, cfg, q, k_cache.cuda(), v.cuda(), [64], 64, cos, sin)
+    assert err.value.status == jl.JL_ERR_UNSUPPORTED
+
+
 def test_decode_replayed_from_a_cuda_graph_follows_the_device_lengths(jl):
     # The decode entry point reads the lengths (and so G) only on the device, so one captured
     # call serves every step: replaying it after the lengths change must give the eager result
@@ -328,8 +387,10 @@ def test_decode_qwen3_4b_cache_lengths(jl, L):
 
 
 def test_decode_walk_across_G_boundary(jl):
-    """Generation across L = 98304 -> 98305 (G 3 -> 4) with no cache rewrite: selected steps of
-    the 256-token walk (positions 98176 .. 98431), all around the boundary."""
+    """Generation across L = 98304 -> 98305 (G 3 -> 4) with no cache rewrite: every one of the
+    256 steps of the walk (query positions 98176 .. 98431) against the oracle.  The cache is
+    rotated once; each step reads its prefix.  The GPU steps run first (each output kept), then
+    the oracle checks them one by one."""
     cfg = I.DECODE_QWEN3_4B
     first, steps = cfg.walk_first_pos, cfg.walk_steps
     max_len = first + steps
@@ -337,13 +398,21 @@ def test_decode_walk_across_G_boundary(jl):
     qs = I.decode_queries(cfg, steps)
     cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
     kd, vd = k_cache.cuda(), v.cuda()
-    chosen = sorted(set(range(124, 132)) | set(range(0, steps, 64)) | {steps - 1})
-    for t in chosen:
+    kbits, vbits = I.bf16_bits(k_cache[0]), I.bf16_bits(v[0])
+    results = []
+    for t in range(steps):
         L = first + t + 1
         q_t = _query_tilde(cfg, qs[t, 0], L)
         out, lse = _run_decode(jl, cfg, q_t[None], kd, vd, [L], max_len, cos, sin)
-        ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
-        _check(out[0], lse[0], ro, rl, f"walk step {t} (L={L}, G={O.group_size(L, cfg.w_pretrained)})")
+        results.append((L, q_t, out[0], lse[0]))
+    groups = set()
+    for t, (L, q_t, out, lse) in enumerate(results):
+        ro, rl = O.decode_step(I.bf16_bits(q_t), kbits[:L], vbits[:L], L, w0=cfg.w0,
+                               w_pretrained=cfg.w_pretrained, rope_base=cfg.rope_base)
+        G = O.group_size(L, cfg.w_pretrained)
+        groups.add(G)
+        _check(out, lse, ro, rl, f"walk step {t} (L={L}, G={G})")
+    assert groups == {3, 4}
 
 
 # ------------------------------------------------- KV cache writers (append) ----

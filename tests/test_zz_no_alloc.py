@@ -60,3 +60,43 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
         assert np.isfinite(got).all(), f"call {call}"
         assert np.abs(got - want).max() <= OUT_MAX, f"call {call}: out differs"
         assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() <= LSE_MAX, f"call {call}: lse differs"
+
+
+@pytest.mark.gpu
+def test_noalloc_decode_head_dim_64_matches_workspace_decode():
+    """head_dim 64 runs the CUDA-core split kernel: two calls in a row (G = 3, then G = 1)."""
+    jl = _lib()
+    from rope_context_extension_sm_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    cfg = I.DecodeConfig("noalloc_d64", (), 8, 2, 64, 100, 1024, 1e4)
+    max_len = 3000
+    k_cache, v = I.decode_raw_inputs(cfg, max_len)
+    kd, vd = k_cache.to(dev), v.to(dev)
+    qs = I.decode_queries(cfg, 2).to(dev)
+    cos, sin = jl.jl_rope_tables(max_len, cfg.head_dim, cfg.rope_base, device=dev)
+    for call, L in enumerate([3000, 700]):
+        sl = torch.tensor([L], dtype=torch.int32, device=dev)
+        q = qs[call].contiguous()
+        ref, ref_lse = jl.jl_bifocal_decode(q, kd, vd, sl, max_len, cfg.w0, cfg.w_pretrained, cos, sin)
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((1, cfg.n_q_heads), float("nan"), dtype=torch.float32, device=dev)
+        jl.jl_bifocal_decode_noalloc(q, kd, vd, sl, max_len, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+        jl.jl_sync_status()
+        got, want = out.float().cpu().numpy(), ref.float().cpu().numpy()
+        assert np.isfinite(got).all(), f"call {call}"
+        assert np.abs(got - want).max() <= OUT_MAX, f"call {call}: out differs"
+        assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() <= LSE_MAX, f"call {call}: lse differs"
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_a_query_outside_device_memory():
+    """The static scratch is only valid on its own device, so the call checks that q is device
+    memory of the current device (and that the stream is that device's) before launching."""
+    jl = _lib()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+    host_q = np.zeros((1, 32, 128), dtype=np.uint16)  # pageable host memory
+    st = jl._lib.jl_bifocal_decode_noalloc(host_q.ctypes.data, 16, 16, 16, 1, 4096, 4096, 32, 8, 128, 64, 1024, 16,
+                                           16, 4096, 0.0, 16, 16, None)
+    assert st == jl.JL_ERR_INVALID
+    assert "not device memory" in jl.jl_last_error()
