@@ -87,8 +87,9 @@ def _source_hash(files):
 PREFILL_SRC = ["rope_context_extension_sm_b200/csrc/jl_prefill.cuh", "rope_context_extension_sm_b200/csrc/jl_device.cuh"]
 
 
-def _traffic(kernel, files):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+def _profiled(kernel, files, key):
+    """A figure from the committed ncu summary (profiles/traffic.txt), if it was taken on this
+    source: DRAM bytes per launch, or the tensor pipe's active fraction."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
             rec = json.load(f).get(kernel)
@@ -96,7 +97,11 @@ def _traffic(kernel, files):
         return None
     if not rec or rec.get("source_hash") != _source_hash(files):
         return None
-    return rec.get("dram_bytes_per_launch")
+    return rec.get(key)
+
+
+def _traffic(kernel, files):
+    return _profiled(kernel, files, "dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -704,6 +709,7 @@ def run_ours(args, world, rank, local):
             "unit": "TFLOP/s",
             "frac": round(prefill_tflops / sustained, 4),
             "traffic": _traffic("prefill", PREFILL_SRC),
+            "tensor_pipe_active": _profiled("prefill", PREFILL_SRC, "tensor_pipe_active_pct"),
             "algorithmic_bytes_per_launch": int(sum(t.numel() * t.element_size() for t in (q, k, v, out, lse))),
         },
         "e2e": {

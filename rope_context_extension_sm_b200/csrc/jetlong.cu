@@ -213,8 +213,43 @@ jl_status prefill_params(const void* q, const void* k, const void* v, const int3
   return ok();
 }
 
+// One query head per CTA with double-buffered scores (jl_prefill_db_kernel).
+template <int D>
+jl_status launch_prefill_db(const void* q, const void* k, const void* v, jl::PrefillParams prm, cudaStream_t st) {
+  using Lay = jl::PrefillDbLayout<D>;
+  prm.slots = prm.group;  // every query head is its own CTA
+  CUtensorMap tq, tk, tv;
+  jl_status s;
+  if ((s = make_map(&tq, q, prm.total_tokens, prm.Hq, D)) != JL_OK) return s;
+  const int64_t kv_rows = prm.cached ? static_cast<int64_t>(prm.batch) * prm.cache_stride : prm.total_tokens;
+  if ((s = make_map(&tk, k, kv_rows, prm.Hkv, D)) != JL_OK) return s;
+  if ((s = make_map(&tv, v, kv_rows, prm.Hkv, D)) != JL_OK) return s;
+  auto kern = jl::jl_prefill_db_kernel<D>;
+  const KernelAttr attr = kernel_attr(reinterpret_cast<const void*>(kern), Lay::kAlloc);
+  if (attr.err != cudaSuccess) return cuda_fail(attr.err, "cudaFuncSetAttribute(prefill)");
+  // the softmax warpgroup's register increase would wait forever if the launch
+  // allocation could not cover the split, so such a build is refused
+  if (static_cast<int64_t>(attr.regs) * Lay::kThreads < Lay::kRegsNeeded)
+    return fail(JL_ERR_UNSUPPORTED, "prefill kernel built with %d registers per thread; the register split needs %u",
+                attr.regs, Lay::kRegsLaunch);
+  const int64_t blocks = static_cast<int64_t>(prm.n_qtiles) * prm.batch * prm.Hkv * prm.slots;
+  if (blocks > 0x7fffffff) return fail(JL_ERR_UNSUPPORTED, "prefill grid too large (%lld blocks)", (long long)blocks);
+  kern<<<static_cast<unsigned>(blocks), Lay::kThreads, Lay::kAlloc, st>>>(tq, tk, tv, prm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return ok();
+}
+
+// JL_PREFILL_DB = 1 routes head_dim 128 to jl_prefill_db_kernel (one head per CTA,
+// double-buffered scores).  It is correct (the GPU suite passes on it) but measured
+// slower than the two-head kernel on the 128K layer, so it is built, not used.
+#ifndef JL_PREFILL_DB
+#define JL_PREFILL_DB 0
+#endif
+
 jl_status launch_prefill_any(const void* q, const void* k, const void* v, const jl::PrefillParams& prm,
                              int32_t head_dim, cudaStream_t st) {
+  if (JL_PREFILL_DB && head_dim == 128) return launch_prefill_db<128>(q, k, v, prm, st);
   const bool pair = (prm.group % 2) == 0;
   if (head_dim == 128)
     return pair ? launch_prefill<128, 2>(q, k, v, prm, st) : launch_prefill<128, 1>(q, k, v, prm, st);

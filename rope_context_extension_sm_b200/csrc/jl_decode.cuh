@@ -61,12 +61,12 @@ template <int D>
 __device__ __forceinline__ void load_half_bf16(const __nv_bfloat16* p, float (&x)[D / 32]) {
   if constexpr (D == 128) {
     const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    const float2 a = unpack_bf16x2(u.x);
+    const float2 b = unpack_bf16x2(u.y);
     x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
   } else {
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+    const float2 a = unpack_bf16x2(u);
     x[0] = a.x; x[1] = a.y;
   }
 }

@@ -13,7 +13,8 @@
 // entry, or a page pool with a block table (pages of a multiple of 128 keys, so a
 // tile lies in one page).  Per 128-key tile:
 //   warp 0      TMA producer: raw K and V tiles (3 stages)
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator + tcgen05.mma issuer (warp-uniform loop, one
+//               elected lane issues, descriptors formed once)
 //   warps 2-3,  correction warps (16, or 8 for 16 heads per KV head): rotate
 //   8..         the remote rows of the K tile in place by R(-(j - f(j)))
 //               (cos/sin stepped along the rows by complex
@@ -90,18 +91,18 @@ __device__ __forceinline__ int dec_rot_index(int warp) {
 __device__ __forceinline__ void rotate_row_neg(uint8_t* tile, int r, const float (&c)[2], const float (&s)[2],
                                                int lane) {
   const int off = r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + ((lane & 3) << 2);
-  __nv_bfloat162* plo = reinterpret_cast<__nv_bfloat162*>(tile + off);
-  __nv_bfloat162* phi = reinterpret_cast<__nv_bfloat162*>(tile + 16384 + off);
-  const float2 a = __bfloat1622float2(*plo);
-  const float2 b = __bfloat1622float2(*phi);
+  uint32_t* plo = reinterpret_cast<uint32_t*>(tile + off);
+  uint32_t* phi = reinterpret_cast<uint32_t*>(tile + 16384 + off);
+  const float2 a = unpack_bf16x2(*plo);
+  const float2 b = unpack_bf16x2(*phi);
   // ya = a c + b s, yb = b c - a s on packed pairs (two frequencies per instruction)
   const uint64_t c2 = f2_pack(c[0], c[1]), s2 = f2_pack(s[0], s[1]);
   const uint64_t a2 = f2_pack(a.x, a.y), b2 = f2_pack(b.x, b.y);
   float2 ya, yb;
   f2_unpack(f2_fma(b2, s2, f2_mul(a2, c2)), ya.x, ya.y);
   f2_unpack(f2_sub(f2_mul(b2, c2), f2_mul(a2, s2)), yb.x, yb.y);
-  *plo = __float22bfloat162_rn(ya);
-  *phi = __float22bfloat162_rn(yb);
+  *plo = pack_bf16x2(ya.x, ya.y);
+  *phi = pack_bf16x2(yb.x, yb.y);
 }
 
 // (c, s) <- (c, s) * e^{i theta} when adv, else unchanged (select, no branch).
@@ -122,9 +123,9 @@ __device__ __forceinline__ void step_factor(float (&c)[2], float (&s)[2], const 
 // Correct the remote rows (r <= last_remote) of an ROWS-row slice of keys j0 ..:
 // R(-n_j), n_j = j - floor(j / G).  n steps by one per row except where f steps up
 // (row r with (j0 + r + 1) % G == 0).  GS = G in {2, 4, 8} with j0 % G == 0 makes
-// those rows compile-time; GS = 0 keeps a counter and selects.
+// those rows compile-time; GS = 0 starts from j0_mod_g = j0 mod G (unused otherwise).
 template <int ROWS, int GS>
-__device__ __forceinline__ void correct_slice(uint8_t* slice, int j0, int G, int last_remote, bool full,
+__device__ __forceinline__ void correct_slice(uint8_t* slice, int j0_mod_g, int G, int last_remote, bool full,
                                               float (&fc)[2], float (&fs)[2], const float (&st_c)[2],
                                               const float (&st_s)[2], int lane) {
   if constexpr (GS > 0) {
@@ -146,7 +147,7 @@ __device__ __forceinline__ void correct_slice(uint8_t* slice, int j0, int G, int
     // (j0 + r + 1) % G == 0), computed once per slice so the row loop carries no
     // counter; the partial-slice test is hoisted out of the loop like above.
     uint32_t adv = 0;
-    int cnt = j0 % G;
+    int cnt = j0_mod_g;
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       cnt = (cnt + 1 == G) ? 0 : cnt + 1;
@@ -252,19 +253,20 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int issued[kDecStages] = {0};
+      StepDiv pdiv{};  // page and row of the tile's first key, stepped per tile (paged caches)
+      if (p.block_table != nullptr) pdiv.init(c0, kDecTile, p.page_size);
       for (int n = 0; n < n_tiles && !*abort; ++n) {
         const int s = n % kDecStages;
         const uint32_t u = n / kDecStages;
         const int kpos = c0 + n * kDecTile;  // key position in entry b; a tile never crosses a page
         const int key0 = p.block_table != nullptr
-                             ? p.block_table[static_cast<int64_t>(b) * p.max_pages + kpos / p.page_size] * p.page_size +
-                                   kpos % p.page_size
+                             ? p.block_table[static_cast<int64_t>(b) * p.max_pages + pdiv.q] * p.page_size + pdiv.r
                              : static_cast<int>(row0) + kpos;
         // contiguous: the tile's keys lie in entry b; paged: its page is inside the pool
         JL_CHECK(kpos < L && (p.block_table != nullptr
-                                  ? (kpos / p.page_size < p.max_pages && key0 >= 0 &&
-                                     key0 + kDecTile <= p.cache_stride)
+                                  ? (pdiv.q < p.max_pages && key0 >= 0 && key0 + kDecTile <= p.cache_stride)
                                   : L <= p.cache_stride));
+        if (p.block_table != nullptr) pdiv.next();
         JL_DTRACE_AT(n, 0);
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         JL_DTRACE_AT(n, 1);
@@ -285,61 +287,70 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-      auto issue_s = [&](int n) {
-        const uint32_t ka = k_addr + (n % kDecStages) * Lay::kTile;
+    // The whole warp runs the loop, so every operand stays warp-uniform, and one
+    // elected lane issues each tcgen05 instruction.  Descriptors are formed once:
+    // the descriptor of (base + off) is that of base plus off / 16 (the start-address
+    // field, which cannot carry below 256 KB of shared memory).
+    const bool leader = elect_one();
+    const uint64_t dk0 = sdesc_kmajor_sw128(smem_u32(sK));
+    const uint64_t dv0 = sdesc_mnmajor_sw128(smem_u32(sV), 16384);
+    const uint64_t dq0 = sdesc_kmajor_sw128(smem_u32(sQ));
+    const uint64_t dp0 = sdesc_kmajor_sw128(smem_u32(sP));
+    auto issue_s = [&](int n) {
+      const uint64_t kd = dk0 + static_cast<uint32_t>(((n % kDecStages) * Lay::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off_k = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t off_q = (kk >> 2) * (kDecQRows * 128) + (kk & 3) * 32;
-          umma_ss(tmem + (n & 1) * 32, sdesc_kmajor_sw128(ka + off_k), sdesc_kmajor_sw128(q_addr + off_q), kIdescS,
-                  kk > 0);
-        }
-      };
-      auto issue_pv = [&](int n) {
-        const uint32_t va = v_addr + (n % kDecStages) * Lay::kTile;
-        const uint32_t pa = p_addr + (n & 1) * (kDecHeads * 256);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off_k = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+        const uint32_t off_q = ((kk >> 2) * (kDecQRows * 128) + (kk & 3) * 32) >> 4;
+        if (leader) umma_ss(tmem + (n & 1) * 32, kd + off_k, dq0 + off_q, kIdescS, kk > 0);
+      }
+    };
+    auto issue_pv = [&](int n) {
+      const uint64_t vd = dv0 + static_cast<uint32_t>(((n % kDecStages) * Lay::kTile) >> 4);
+      const uint64_t pd = dp0 + static_cast<uint32_t>(((n & 1) * (kDecHeads * 256)) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off_p = (kk >> 2) * (kDecHeads * 128) + (kk & 3) * 32;
-          umma_ss(tmem + 64, sdesc_mnmajor_sw128(va + kk * 2048, 16384), sdesc_kmajor_sw128(pa + off_p), kIdescO,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(&bars->q_ready, 0, abort);
-      if (ok) {
-        tc_fence_after();
-        ok = mbar_wait(&bars->k_ready[0], 0, abort);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off_p = ((kk >> 2) * (kDecHeads * 128) + (kk & 3) * 32) >> 4;
+        if (leader) umma_ss(tmem + 64, vd + ((kk * 2048) >> 4), pd + off_p, kIdescO, (n > 0 || kk > 0) ? 1u : 0u);
       }
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        umma_commit(&bars->s_full[0]);
-        umma_commit(&bars->k_empty[0]);
-      }
-      for (int n = 0; n < n_tiles && ok; ++n) {
-        if (n + 1 < n_tiles) {  // scores of the next tile overlap this tile's softmax
-          const int s1 = (n + 1) % kDecStages;
-          if (!(ok = mbar_wait(&bars->k_ready[s1], ((n + 1) / kDecStages) & 1, abort))) break;
-          tc_fence_after();
-          issue_s(n + 1);
-          JL_DTRACE_AT(n + 1, 5);
-          umma_commit(&bars->s_full[(n + 1) & 1]);
-          umma_commit(&bars->k_empty[s1]);
-        }
-        if (!(ok = mbar_wait(&bars->p_ready[n & 1], (n >> 1) & 1, abort))) break;
-        tc_fence_after();
-        const int s = n % kDecStages;
-        if (!(ok = mbar_wait(&bars->v_full[s], (n / kDecStages) & 1, abort))) break;
-        JL_DTRACE_AT(n, 4);
-        issue_pv(n);
-        umma_commit(&bars->pv_done);
-        umma_commit(&bars->v_empty[s]);
-      }
-      umma_commit(&bars->teardown);
-      mbar_wait_bounded(&bars->teardown, 0);
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) umma_commit(bar);
+    };
+    bool ok = warp_wait(&bars->q_ready, 0, abort);
+    if (ok) {
+      tc_fence_after();
+      ok = warp_wait(&bars->k_ready[0], 0, abort);
     }
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+      commit(&bars->s_full[0]);
+      commit(&bars->k_empty[0]);
+    }
+    for (int n = 0; n < n_tiles && ok; ++n) {
+      if (n + 1 < n_tiles) {  // scores of the next tile overlap this tile's softmax
+        const int s1 = (n + 1) % kDecStages;
+        if (!(ok = warp_wait(&bars->k_ready[s1], ((n + 1) / kDecStages) & 1, abort))) break;
+        tc_fence_after();
+        issue_s(n + 1);
+        JL_DTRACE_AT(n + 1, 5);
+        commit(&bars->s_full[(n + 1) & 1]);
+        commit(&bars->k_empty[s1]);
+      }
+      if (!(ok = warp_wait(&bars->p_ready[n & 1], (n >> 1) & 1, abort))) break;
+      tc_fence_after();
+      const int s = n % kDecStages;
+      if (!(ok = warp_wait(&bars->v_full[s], (n / kDecStages) & 1, abort))) break;
+      JL_DTRACE_AT(n, 4);
+      issue_pv(n);
+      commit(&bars->pv_done);
+      commit(&bars->v_empty[s]);
+    }
+    // Every issued MMA must finish before TMEM is released.
+    commit(&bars->teardown);
+    mbar_wait_bounded(&bars->teardown, 0);
+    __syncwarp();
   } else if (dec_rot_index(warp) >= 0) {
     // ---------------------------------------------------- correction warps
     const int rw = dec_rot_index(warp);
@@ -349,9 +360,16 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       const float2 ss = __ldg(reinterpret_cast<const float2*>(p.sin_tab + 64 + 2 * lane));
       st_c[0] = cc.x; st_c[1] = cc.y; st_s[0] = ss.x; st_s[1] = ss.y;
     }
-    auto anchor = [&](int n, float (&c)[2], float (&s)[2]) {
+    // j / G for this warp's first key, stepped from tile to tile (one division here;
+    // a division per tile would queue on the MUFU unit behind the softmax).
+    StepDiv jdiv{};
+    if (G > 1) jdiv.init(c0 + Lay::kRotRows * rw, kDecTile, G);
+    // anchor of tile n (called for n = 0, 1, 2, ... in order); rem = j mod G of its first key
+    auto anchor = [&](int n, float (&c)[2], float (&s)[2], int& rem) {
       const int j = c0 + n * kDecTile + Lay::kRotRows * rw;
-      int64_t row = j - j / G;  // correction index n_j = j - f(j)
+      int64_t row = G > 1 ? j - jdiv.q : 0;  // correction index n_j = j - f(j)
+      rem = G > 1 ? jdiv.r : 0;
+      if (G > 1) jdiv.next();
       {
         const int last = min(j + Lay::kRotRows - 1, c1 - 1);  // rows of the valid keys of this slice
         JL_CHECK(j > last || last - last / G < p.n_tab_rows);
@@ -362,10 +380,12 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       c[0] = cc.x; c[1] = cc.y; s[0] = ss.x; s[1] = ss.y;
     };
     float nc[2], ns[2];
-    anchor(0, nc, ns);
+    int nrem = 0;
+    anchor(0, nc, ns, nrem);
     for (int n = 0; n < n_tiles; ++n) {
       float fc[2] = {nc[0], nc[1]}, fs[2] = {ns[0], ns[1]};
-      if (n + 1 < n_tiles) anchor(n + 1, nc, ns);
+      const int rem = nrem;
+      if (n + 1 < n_tiles) anchor(n + 1, nc, ns, nrem);
       const int s = n % kDecStages;
       if (!mbar_wait(&bars->k_full[s], (n / kDecStages) & 1, abort)) break;
       if (rw == 0) JL_DTRACE_AT(n, 2);
@@ -378,7 +398,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
           case 2: correct_slice<Lay::kRotRows, 2>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
           case 4: correct_slice<Lay::kRotRows, 4>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
           case 8: correct_slice<Lay::kRotRows, 8>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
-          default: correct_slice<Lay::kRotRows, 0>(slice, j0, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
+          default: correct_slice<Lay::kRotRows, 0>(slice, rem, G, last_remote, full, fc, fs, st_c, st_s, lane); break;
         }
         fence_proxy_async_smem();
       }
@@ -473,7 +493,7 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
         const float m_use = (m_run[g] == -INFINITY) ? 0.f : m_run[g];
         const float pr = valid ? ex2_approx(fmaf(sv[g], sl2, -m_use)) : 0.f;
         l_part[g] = l_part[g] * alpha[g] + pr;
-        *reinterpret_cast<__nv_bfloat16*>(pb + swz_off(g, tid, kDecHeads * 128)) = __float2bfloat16_rn(pr);
+        *reinterpret_cast<uint16_t*>(pb + swz_off(g, tid, kDecHeads * 128)) = pack_bf16(pr);
       }
       if (any_resc && n > 0) {  // uniform: every thread computed the same alphas
         uint32_t o[32];

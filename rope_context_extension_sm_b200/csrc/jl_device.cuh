@@ -64,22 +64,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Arrive that cannot be issued before `dep` is computed: the value is an input of
-// the instruction, so every operation feeding it (e.g. a row sum over the
-// exponentials) completes first.
-__device__ __forceinline__ void mbar_arrive_after(uint64_t* bar, float dep) {
-  asm volatile("{\n .reg .f32 d;\n mov.b32 d, %1;\n mbarrier.arrive.shared::cta.b64 _, [%0];\n}\n" ::"r"(smem_u32(bar)),
-               "f"(dep)
-               : "memory");
-}
-
-// Returns x through an opaque move, so work that uses the result is not started
-// before the preceding (volatile) instructions, e.g. a barrier wait.
-__device__ __forceinline__ float order_after(float x) {
-  asm volatile("mov.b32 %0, %0;" : "+f"(x)::"memory");
-  return x;
-}
-
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
@@ -362,22 +346,47 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Two finite floats to a bf16 pair on the integer pipe: half a bf16 ulp is added
-// to each bit pattern (rounding the magnitude to nearest, ties away from zero)
-// and the two upper halves are byte-permuted together.  Differs from the
-// round-to-nearest-even conversion only on exact ties.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
-#ifndef JL_IPACK
-#define JL_IPACK 0  // 1: P packed on the integer pipe; 2: the rotations' outputs too
+// bf16 <-> fp32 in the hot loops.  The conversion instructions run on the same
+// unit as the MUFU exponentials the softmax depends on, so with JL_ALUCVT the
+// conversions are done on the integer pipe instead: a bf16 is the upper half of
+// the fp32 of the same value, so widening is a shift or a mask (exact); narrowing
+// rounds to nearest even by adding 0x7fff plus the lowest kept bit, for finite
+// values (as the conversion does).  1: widening only; 2: both directions.
+#ifndef JL_ALUCVT
+#define JL_ALUCVT 1
 #endif
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  if constexpr (JL_ALUCVT >= 1) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  } else {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  if constexpr (JL_ALUCVT >= 2) {
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a += 0x7fffu + ((a >> 16) & 1u);
+    b += 0x7fffu + ((b >> 16) & 1u);
+    return __byte_perm(a, b, 0x7632);
+  } else {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// One value, as the low 16 bits (same rounding as pack_bf16x2).
+__device__ __forceinline__ uint16_t pack_bf16(float x) {
+  if constexpr (JL_ALUCVT >= 2) {
+    uint32_t a = __float_as_uint(x);
+    a += 0x7fffu + ((a >> 16) & 1u);
+    return static_cast<uint16_t>(a >> 16);
+  } else {
+    const __nv_bfloat16 v = __float2bfloat16_rn(x);
+    return *reinterpret_cast<const uint16_t*>(&v);
+  }
+}
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
@@ -404,6 +413,29 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// floor(x / d) and x mod d for an x that advances by a fixed step: one division
+// at init, additions after.  (Integer division by a value known only at run time
+// issues reciprocal instructions on the MUFU unit, where they would queue behind
+// the softmax's exponentials.)  Requires 0 <= x, step and d >= 1.
+struct StepDiv {
+  int q, r, dq, dr, d;
+  __device__ __forceinline__ void init(int x, int step, int div) {
+    d = div;
+    q = x / d;
+    r = x - q * d;
+    dq = step / d;
+    dr = step - dq * d;
+  }
+  __device__ __forceinline__ void next() {
+    q += dq;
+    r += dr;
+    if (r >= d) {
+      r -= d;
+      ++q;
+    }
+  }
+};
 
 // One lane of the (converged) warp is elected; the others get false.
 __device__ __forceinline__ bool elect_one() {
