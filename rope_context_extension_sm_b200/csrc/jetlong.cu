@@ -240,17 +240,20 @@ jl_status launch_prefill_db(const void* q, const void* k, const void* v, jl::Pre
   return ok();
 }
 
-// JL_PREFILL_DB = 1 routes head_dim 128 to jl_prefill_db_kernel (one head per CTA,
-// double-buffered scores).  It is correct (the GPU suite passes on it) but measured
-// slower than the two-head kernel on the 128K layer, so it is built, not used.
+// Which kernel: an even GQA group pairs two query heads per CTA (jl_prefill_kernel
+// <D, 2>: one K/V tile and one rotation serve both).  An odd group (multi-head
+// attention included) has a head with no partner; at head_dim 128 it runs one head
+// per CTA with double-buffered scores (jl_prefill_db_kernel), about 1.3x the
+// single-buffered one-head kernel on those shapes.  JL_PREFILL_DB = 1 at build time
+// sends every head_dim-128 call there (for measurements).
 #ifndef JL_PREFILL_DB
 #define JL_PREFILL_DB 0
 #endif
 
 jl_status launch_prefill_any(const void* q, const void* k, const void* v, const jl::PrefillParams& prm,
                              int32_t head_dim, cudaStream_t st) {
-  if (JL_PREFILL_DB && head_dim == 128) return launch_prefill_db<128>(q, k, v, prm, st);
   const bool pair = (prm.group % 2) == 0;
+  if (head_dim == 128 && (JL_PREFILL_DB || !pair)) return launch_prefill_db<128>(q, k, v, prm, st);
   if (head_dim == 128)
     return pair ? launch_prefill<128, 2>(q, k, v, prm, st) : launch_prefill<128, 1>(q, k, v, prm, st);
   return pair ? launch_prefill<64, 2>(q, k, v, prm, st) : launch_prefill<64, 1>(q, k, v, prm, st);

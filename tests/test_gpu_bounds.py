@@ -40,7 +40,8 @@ def jlb():
 
 
 @pytest.mark.parametrize("name", ["gqa4_G4_w0_100", "gqa4_G4_w0_0", "w0_covers_all", "G1_short", "varlen_ragged",
-                                  "group3_d64", "d64_gqa2"])
+                                  "group3_d64", "d64_gqa2", "group3_d128_G4", "group3_d128_varlen",
+                                  "group1_d128_w0_0"])
 def test_bounds_build_prefill(jlb, name):
     case = next(c for c in P.SMALL if c[0] == name)
     _, seqlens, hq, hkv, d, w0, w_pre = case
@@ -60,6 +61,7 @@ def test_bounds_build_prefill_and_cache(jlb, case):
 def test_bounds_build_chunked_three_pass_interp(jlb):
     P.test_chunked_prefill_single_sequence_across_G(jlb)
     P.test_chunked_prefill_d64_group3(jlb)
+    P.test_chunked_prefill_d128_group3(jlb)
     P.test_three_pass_merge_on_gpu(jlb, P.THREE_PASS[0])
     P.test_interp_prefill_matches_oracle(jlb, P.INTERP[1])
 

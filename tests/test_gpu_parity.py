@@ -131,6 +131,12 @@ SMALL = [
     ("varlen_ragged", (1, 130, 257, 700, 64, 129), 4, 2, 128, 50, 128),
     ("group3_d64", (500,), 3, 1, 64, 40, 100),
     ("group1_d128", (384,), 2, 2, 128, 64, 100),
+    # odd groups at head_dim 128 run the one-head double-buffered kernel
+    ("group3_d128_G4", (1000,), 6, 2, 128, 100, 256),
+    ("group1_d128_G5_w0_129", (600,), 3, 3, 128, 129, 128),
+    ("group3_d128_varlen", (1, 130, 257, 700, 0, 64), 3, 1, 128, 50, 128),
+    ("group1_d128_w0_0", (500,), 2, 2, 128, 0, 128),
+    ("group3_d128_w0_covers", (300,), 3, 1, 128, 5000, 100),
     ("d64_gqa2", (450,), 4, 2, 64, 33, 64),
 ]
 
@@ -445,6 +451,8 @@ PREFILL_AND_CACHE = [
     ("G1_plain", (200,), 4, 2, 128, 32, 256),
     ("w0_0_writer_fallback", (300,), 4, 2, 128, 0, 64),
     ("d64_group3", (257, 70), 3, 1, 64, 16, 64),
+    ("d128_group3", (257, 700), 3, 1, 128, 16, 64),
+    ("d128_group1_w0_0", (300,), 2, 2, 128, 0, 64),
 ]
 
 
@@ -525,6 +533,7 @@ THREE_PASS = [
     ("tp_varlen", (1, 130, 257, 700, 0, 64), 4, 2, 128, 50, 128),
     ("tp_w0_covers", (400,), 2, 2, 128, 5000, 100),
     ("tp_d64_group3", (500,), 3, 1, 64, 40, 100),
+    ("tp_d128_group3", (700,), 3, 1, 128, 100, 256),
 ]
 
 
@@ -621,6 +630,11 @@ def test_chunked_prefill_d64_group3(jl):
     _chunked_run(jl, "chunk_d64", [500], [[129], [371]], 3, 1, 64, 40, 100)
 
 
+def test_chunked_prefill_d128_group3(jl):
+    # odd group at head_dim 128: the one-head double-buffered kernel with cached keys
+    _chunked_run(jl, "chunk_d128_g3", [900, 300], [[130, 0], [400, 300], [370, 0]], 3, 1, 128, 64, 200)
+
+
 # --------------------------------------------------------------- paged caches ----
 
 def _paginate(cache, lens, page_size, seed=3):
@@ -713,6 +727,7 @@ INTERP = [
     ("yarn_s4", (1000,), 8, 2, 128, 100, "yarn", 4.0),
     ("yarn_varlen", (300, 129, 700), 4, 2, 128, 64, "yarn", 3.0),
     ("pi_d64_w0_0", (400,), 3, 1, 64, 0, "pi", 2.0),
+    ("yarn_d128_group3", (600, 129), 3, 1, 128, 64, "yarn", 4.0),
 ]
 
 
