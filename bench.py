@@ -719,7 +719,7 @@ def run_ours(args, world, rank, local):
             "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h),
         },
-        "gpu_launches": 3 * K,
+        "gpu_launches": 3 * K,  # per step: the prefill kernel, the decode split kernel and its merge
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:

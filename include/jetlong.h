@@ -79,6 +79,18 @@ jl_status jl_sync_status(jl_stream_t stream);
 int jl_debug_bounds_enabled(void);
 
 /*
+ * Single-launch decode build (no counterpart in the paper; a variant of this
+ * library).  Returns 1 in the library built with -DJL_DECODE_LAST_CTA_MERGE=1
+ * (libjetlong_lastcta.so), 0 otherwise.  In that build the head_dim-128 decode is
+ * one kernel launch: the last split CTA of each (entry, KV head) merges the split
+ * partials (see jl_bifocal_decode).  The normal build merges them in a second,
+ * small kernel, which measured faster on B200: the last CTA's atomic ticket and
+ * its reads of the other CTAs' partials are serial L2 round trips that cost more
+ * than the kernel boundary they save.
+ */
+int jl_decode_single_launch_enabled(void);
+
+/*
  * Failure-detection self-test (no counterpart in the paper; it exercises this
  * library's bounded waits).  Launches one thread that waits on a shared-memory
  * barrier that nothing ever completes, giving up after limit_cycles SM clock
@@ -255,6 +267,17 @@ jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const in
  *   workspace    device scratch of at least jl_bifocal_decode_workspace_size()
  *                bytes, 16-byte aligned, owned by the caller; its contents on
  *                entry do not matter; calls sharing it must not overlap.
+ * The keys are split across CTAs; a second, small kernel merges the split
+ * partials.  In the single-launch build (jl_decode_single_launch_enabled) the
+ * head_dim-128 call is one kernel launch instead: the last CTA of each (entry,
+ * KV head) to finish merges them.  It is found through two counter words per
+ * (entry, KV head) in the workspace: a count that the last CTA puts back to a
+ * marked zero, and, for a workspace whose count word is not marked yet, a second
+ * count tagged with a value unique to the call (a word with another tag counts
+ * as zero).  So the workspace needs no clearing in either build, and a CUDA
+ * graph replaying the call finds the count clear.  A CTA that gives up on a
+ * bounded wait still counts.  In both builds out and lse are written as NaN when
+ * a kernel of the call gave up.
  * Local keys (i - j < w0) score q . k_cache[j] unchanged; remote keys score
  * (R(f(i) - i) q) . (R(f(j) - j) k_cache[j]), both corrections applied in
  * registers.  G = max(1, ceil(seqlens[b] / w_pretrained)) is computed on the
@@ -353,7 +376,8 @@ jl_status jl_decode_append_paged(const void* q, const void* k, const void* v, co
  * device array of jl_bifocal_decode_noalloc_scratch_bytes() bytes (8 MiB) that
  * every GPU loading the library holds until the process exits.
  *  - Sizes whose scratch would exceed that maximum (B * n_split * Hq *
- *    (head_dim + 2) * 4 bytes, see jl_bifocal_decode_workspace_size) return
+ *    (head_dim + 2) * 4 bytes of partials plus B * Hq * 16 bytes of merge
+ *    counters, see jl_bifocal_decode_workspace_size) return
  *    JL_ERR_INVALID with a message; B = 1, Hq = 32, head_dim = 128 fits up to
  *    max_seqlen = 131072.
  *  - The stream, the current device and q must be on one device; a mismatch

@@ -54,6 +54,16 @@ def build_bounds(force: bool = False) -> str:
     return build(force=force, extra=["-DJL_DEBUG_BOUNDS"], out=BOUNDS_LIB)
 
 
+# The single-launch decode build: the last split CTA of each (entry, KV head) merges
+# the partials instead of a second kernel (-DJL_DECODE_LAST_CTA_MERGE=1).
+LAST_CTA_LIB = os.path.join(HERE, "libjetlong_lastcta.so")
+
+
+def build_last_cta(force: bool = False) -> str:
+    """Build libjetlong_lastcta.so (the single-launch decode variant) in-tree."""
+    return build(force=force, extra=["-DJL_DECODE_LAST_CTA_MERGE=1"], out=LAST_CTA_LIB)
+
+
 if __name__ == "__main__":
     build(force=True, verbose=True, extra=sys.argv[1:])
     print(LIB)

@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <string>
@@ -328,8 +329,10 @@ jl_status launch_decode_tc(const jl::DecodeParams& prm, int B, cudaStream_t st) 
   dim3 grid(prm.Hkv, prm.n_split, B);
   cudaError_t e = launch_pdl(kern, grid, dim3(Lay::kThreads), Lay::kAlloc, st, tk, tv, prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  e = launch_pdl(jl::jl_decode_combine_kernel<128>, dim3(prm.Hq, B), dim3(jl::kCombineThreads), 0, st, prm);
-  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  if (prm.counters == nullptr) {  // no merge counters: a second kernel merges the splits
+    e = launch_pdl(jl::jl_decode_combine_kernel<128>, dim3(prm.Hq, B), dim3(jl::kCombineThreads), 0, st, prm);
+    if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  }
   return ok();
 }
 
@@ -363,9 +366,32 @@ jl_status dispatch_group(const jl::DecodeParams& prm, int B, cudaStream_t st) {
   }
 }
 
-size_t ws_bytes_for(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen, int chunk) {
+// Workspace: the split partials [B][n_split][Hq][head_dim + 2] floats, then (from a
+// 256-byte boundary) two 8-byte merge counter words per (entry, KV head), B * Hq
+// pairs at most.
+size_t partials_bytes(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen, int chunk) {
   const int64_t n_split = (max_seqlen + chunk - 1) / chunk;
-  return static_cast<size_t>(B) * n_split * Hq * (head_dim + 2) * sizeof(float);
+  const size_t n = static_cast<size_t>(B) * n_split * Hq * (head_dim + 2) * sizeof(float);
+  return (n + 255) / 256 * 256;
+}
+
+size_t ws_bytes_for(int32_t B, int32_t Hq, int32_t head_dim, int32_t max_seqlen, int chunk) {
+  return partials_bytes(B, Hq, head_dim, max_seqlen, chunk) + static_cast<size_t>(B) * Hq * 2 * sizeof(uint64_t);
+}
+
+// The head_dim-128 decode merges the split partials in a second kernel unless built
+// with JL_DECODE_LAST_CTA_MERGE = 1, where the last split CTA of each (entry, KV head)
+// merges them in the same launch (measured slower on B200, kept as a tested variant).
+#ifndef JL_DECODE_LAST_CTA_MERGE
+#define JL_DECODE_LAST_CTA_MERGE 0
+#endif
+
+// Tag of one decode call for its merge counters (never 0, the tag of a cleared
+// word).  Successive calls get distinct tags for 2^32 - 1 calls.
+uint32_t next_decode_tag() {
+  static std::atomic<uint32_t> tag{0x5bd1e995u};
+  uint32_t t = tag.fetch_add(1u, std::memory_order_relaxed) + 1u;
+  return t != 0u ? t : tag.fetch_add(1u, std::memory_order_relaxed) + 1u;
 }
 
 // Upper bound over both decode kernels and every KV-head count the query heads
@@ -432,8 +458,14 @@ jl_status decode_common(const void* q, const void* k_cache, const void* v_cache,
   prm.w0 = w0;
   prm.w_pre = w_pretrained;
   prm.plain = plain;
-  prm.chunk = decode_uses_tc(head_dim, Hq, Hkv) ? chunk_tc(B, Hkv, max_seqlen) : chunk_cuda_core(max_seqlen);
+  const bool tc = decode_uses_tc(head_dim, Hq, Hkv);
+  prm.chunk = tc ? chunk_tc(B, Hkv, max_seqlen) : chunk_cuda_core(max_seqlen);
   prm.n_split = (max_seqlen + prm.chunk - 1) / prm.chunk;
+  if (tc && JL_DECODE_LAST_CTA_MERGE) {  // the tensor-core kernel merges in its last CTA per (entry, KV head)
+    prm.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
+                                                         partials_bytes(B, Hq, head_dim, max_seqlen, prm.chunk));
+    prm.epoch = next_decode_tag();
+  }
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(head_dim));
   prm.scale_log2 = scale * 1.4426950408889634f;
   if (head_dim == 128)
@@ -506,6 +538,8 @@ int64_t jl_group_size(int64_t L, int64_t w_pretrained) {
   const int64_t g = (L + w_pretrained - 1) / w_pretrained;
   return g < 1 ? 1 : g;
 }
+
+int jl_decode_single_launch_enabled(void) { return JL_DECODE_LAST_CTA_MERGE ? 1 : 0; }
 
 int jl_debug_bounds_enabled(void) {
 #ifdef JL_DEBUG_BOUNDS
@@ -910,10 +944,10 @@ jl_status jl_bifocal_decode_noalloc(const void* q, const void* k_cache, const vo
   void* scratch = nullptr;
   const jl_status s = static_scratch_for(st, q, &scratch);
   if (s != JL_OK) return s;
-  // Every partial the combine step reads is written earlier in the same call, so
-  // nothing in the scratch needs clearing between calls.  If a split gives up (the
-  // device status word is set), the combine step writes NaN instead of blending
-  // stale partials.
+  // Every partial the merge reads is written earlier in the same call, and the merge
+  // counters count a word with another call's tag as zero, so nothing in the scratch
+  // needs clearing between calls.  If a split gives up (the device status word is
+  // set), the merge writes NaN instead of blending stale partials.
   return decode_common(q, k_cache, v_cache, seqlens, B, cache_stride, max_seqlen, Hq, Hkv, head_dim, w0,
                        w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, scratch,
                        kStaticScratchBytes, st);

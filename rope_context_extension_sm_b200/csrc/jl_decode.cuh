@@ -44,6 +44,10 @@ struct DecodeParams {
   int32_t w0, w_pre, plain;
   int32_t chunk, n_split;
   float scale_log2;
+  // Tensor-core decode only: two words per (entry, KV head) for the last-CTA merge
+  // (null: jl_decode_combine_kernel merges), and this call's tag for those words.
+  unsigned long long* counters;
+  uint32_t epoch;
 };
 
 template <int H>
@@ -287,56 +291,84 @@ __global__ void __launch_bounds__(kCombineThreads) jl_decode_combine_kernel(cons
   constexpr int NW = kCombineThreads / 32;
   const int qh = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();  // the next kernel may set itself up; it waits for this grid before reading
   griddep_wait();  // launched while the split kernel runs: its partials are complete from here on
-  if (status_failed()) {  // a split gave up: its partials are stale, so the output is marked undefined
-    for (int c = threadIdx.x; c < D; c += kCombineThreads) {
-      p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(__int_as_float(0x7fc00000));
-      if (c == 0 && p.lse != nullptr) p.lse[static_cast<int64_t>(b) * p.Hq + qh] = __int_as_float(0x7fc00000);
-    }
-    return;
-  }
+  // The status word, the length and the first batch of partials are loaded together (one
+  // round trip); splits past the length are masked once it is known.
+  const unsigned status = *reinterpret_cast<volatile unsigned*>(&g_status);
   const int L = p.seqlens[b];
   const int ns = (L + p.chunk - 1) / p.chunk;
-  JL_CHECK(L >= 1 && ns <= p.n_split);
   const float* base = p.ws + (static_cast<int64_t>(b) * p.n_split * p.Hq + qh) * (D + 2);
   const int64_t sstride = static_cast<int64_t>(p.Hq) * (D + 2);
-  __shared__ float sm_red[NW], sm_l[NW];
+  __shared__ float sm_m[NW], sm_l[NW];
   __shared__ float sm_o[NW][D];
-  float mx = -INFINITY;
-  for (int s = threadIdx.x; s < ns; s += kCombineThreads) mx = fmaxf(mx, base[s * sstride]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) sm_red[warp] = mx;
-  __syncthreads();
-  float M = sm_red[0];
-#pragma unroll
-  for (int w = 1; w < NW; ++w) M = fmaxf(M, sm_red[w]);
-  float l = 0.f, acc[CPL];
+  // One pass: warp w blends splits w, w + NW, ... with a running maximum (their loads
+  // all in flight together), then the warps' blends are joined in shared memory.
+  constexpr int kBatch = 4;
+  float M = -INFINITY, l = 0.f, acc[CPL];
 #pragma unroll
   for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-  for (int s = warp; s < ns; s += NW) {
-    const float* ps = base + s * sstride;
-    const float ms = ps[0];
-    const float sc = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
-    l = fmaf(ps[1], sc, l);
+  for (int s0 = warp; s0 < p.n_split; s0 += kBatch * NW) {
+    float ms[kBatch], ls[kBatch], os[kBatch][CPL];
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) acc[e] = fmaf(ps[2 + lane * CPL + e], sc, acc[e]);
+    for (int u = 0; u < kBatch; ++u) {  // past n_split: split s0 again; past ns: masked below
+      const int s = s0 + u * NW < p.n_split ? s0 + u * NW : s0;
+      const float* ps = base + s * sstride;
+      ms[u] = ps[0];
+      ls[u] = ps[1];
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) os[u][e] = ps[2 + lane * CPL + e];
+    }
+    if (s0 >= ns) break;
+    bool valid[kBatch];
+    float mb = M;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      valid[u] = s0 + u * NW < ns && ms[u] != -INFINITY;
+      if (valid[u]) mb = fmaxf(mb, ms[u]);
+    }
+    if (mb == -INFINITY) continue;
+    const float r = (M == -INFINITY) ? 0.f : ex2_approx(M - mb);
+    l *= r;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] *= r;
+    M = mb;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (!valid[u]) continue;  // a stale split past the length may hold anything
+      const float sc = ex2_approx(ms[u] - M);
+      l = fmaf(ls[u], sc, l);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[e] = fmaf(os[u][e], sc, acc[e]);
+    }
   }
+  JL_CHECK(L >= 1 && ns <= p.n_split);
 #pragma unroll
   for (int e = 0; e < CPL; ++e) sm_o[warp][lane * CPL + e] = acc[e];
-  if (lane == 0) sm_l[warp] = l;
+  if (lane == 0) {
+    sm_m[warp] = M;
+    sm_l[warp] = l;
+  }
   __syncthreads();
-  float lsum = 0.f;
+  float Mx = sm_m[0];
 #pragma unroll
-  for (int w = 0; w < NW; ++w) lsum += sm_l[w];
+  for (int w = 1; w < NW; ++w) Mx = fmaxf(Mx, sm_m[w]);
+  float sc[NW], lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    sc[w] = (sm_m[w] == -INFINITY) ? 0.f : ex2_approx(sm_m[w] - Mx);
+    lsum = fmaf(sm_l[w], sc[w], lsum);
+  }
+  // a split gave up: its partials are stale, so the output is marked undefined
+  const bool bad = (status & kDevErrTimeout) != 0;
+  const float nan = __int_as_float(0x7fc00000);
   for (int c = threadIdx.x; c < D; c += kCombineThreads) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) o += sm_o[w][c];
-    p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(o / lsum);
+    for (int w = 0; w < NW; ++w) o = fmaf(sm_o[w][c], sc[w], o);
+    p.out[(static_cast<int64_t>(b) * p.Hq + qh) * D + c] = __float2bfloat16_rn(bad ? nan : o / lsum);
     if (c == 0 && p.lse != nullptr)
-      p.lse[static_cast<int64_t>(b) * p.Hq + qh] = (M + log2f(lsum)) * 0.69314718055994531f;
+      p.lse[static_cast<int64_t>(b) * p.Hq + qh] = bad ? nan : (Mx + log2f(lsum)) * 0.69314718055994531f;
   }
 }
 

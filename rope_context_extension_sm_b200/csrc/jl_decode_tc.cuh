@@ -26,7 +26,9 @@
 // that straddles the window edge needs no second visit.  Per-head maxima are
 // reduced across the 128 threads each tile; row sums stay per thread and are
 // reduced once at the end.  The partial (m, l, o) per query head goes to the
-// workspace; jl_decode_combine_kernel merges the splits.
+// workspace.  With p.counters set, the last CTA of each (entry, KV head) to finish
+// merges that head group's partials itself (one launch per decode); otherwise
+// jl_decode_combine_kernel merges them.
 #pragma once
 
 #include "jl_decode.cuh"
@@ -78,9 +80,141 @@ struct DecTcBars {
   uint64_t v_full[kDecStages], v_empty[kDecStages];
   uint64_t s_full[2], p_ready[2], pv_done, q_ready, teardown;
   uint64_t red_full[2], red_end;  // softmax-warp exchanges (bounded, unlike bar.sync)
+  uint64_t fin;                   // the partials of every softmax thread are written
   uint32_t tmem_base;
   int abort;
+  int last;                       // this CTA merges its head group's partials
 };
+
+// Ticket of one split CTA of an (entry, KV head): true for the last of its n CTAs.
+// Two 8-byte words per (entry, KV head), neither of which has to start cleared:
+//  - words[0] holds (kTicketClean << 32) | count once in use.  Each CTA adds 1 (one
+//    atomic, no retries); the one that finds count n - 1 is last and puts the word
+//    back to (kTicketClean, 0) -- every add of the call is in by then -- so the next
+//    call, or a graph replaying this one, finds it clear.
+//  - A words[0] without the marker (a workspace never used by a decode) sends every
+//    CTA of the call (all of them add to the same unmarked word) to words[1].  That
+//    word holds (tag << 32) | count, tag = the call's p.epoch, and a word with another
+//    tag counts as zero; it is advanced by compare-and-swap, bounded since each failed
+//    exchange means another CTA's succeeded.  Its last CTA marks words[0].
+// The atomics are acquire-release at GPU scope: they publish every store the calling
+// thread has observed (the CTA's partials, ordered before it by an mbarrier) and, for
+// the last CTA, make the other CTAs' partials visible.
+constexpr uint32_t kTicketClean = 0x4a4c3136u;
+constexpr unsigned long long kTicketCleanWord = static_cast<unsigned long long>(kTicketClean) << 32;
+
+__device__ __forceinline__ unsigned long long add_acq_rel(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ unsigned long long cas_acq_rel(unsigned long long* p, unsigned long long cmp,
+                                                          unsigned long long val) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;" : "=l"(old) : "l"(p), "l"(cmp), "l"(val)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void store_relaxed(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ bool take_ticket(unsigned long long* words, uint32_t tag, int n) {
+  const unsigned long long old = add_acq_rel(words, 1ull);
+  if (static_cast<uint32_t>(old >> 32) == kTicketClean) {
+    const bool last = static_cast<uint32_t>(old) + 1u >= static_cast<uint32_t>(n);
+    if (last) store_relaxed(words, kTicketCleanWord);
+    return last;
+  }
+  unsigned long long cur;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(cur) : "l"(words + 1) : "memory");
+  for (int tries = 0; tries < 4 * n + 64; ++tries) {
+    const uint32_t cnt = (static_cast<uint32_t>(cur >> 32) == tag) ? static_cast<uint32_t>(cur) + 1u : 1u;
+    const bool last = cnt >= static_cast<uint32_t>(n);
+    const unsigned long long want = (static_cast<unsigned long long>(tag) << 32) | (last ? 0u : cnt);
+    const unsigned long long seen = cas_acq_rel(words + 1, cur, want);
+    if (seen == cur) {
+      if (last) store_relaxed(words, kTicketCleanWord);
+      return last;
+    }
+    cur = seen;
+  }
+  atomicOr(&g_status, kDevErrTimeout);
+  return false;
+}
+
+// Merge of the ns split partials of query heads [hk * ng, hk * ng + ng) of entry b,
+// by all nthreads threads of the last CTA.  The same log-sum-exp blend as
+// jl_decode_combine_kernel.  Item = (head, channel pair); lanes l and l ^ 16 of a warp
+// take the first and the second half of the splits, each with a running maximum, and
+// join through a shuffle, so up to 2 * kMergeBatch splits take one round of loads.
+// Partials written by other CTAs in this launch are read through L2 (ld.global.cg).
+constexpr int kMergeBatch = 8;
+__device__ __forceinline__ void merge_head_group(const DecodeParams& p, int b, int hk, int ng, int ns,
+                                                 int nthreads, bool failed) {
+  // A CTA that gave up set the status word before its ticket, so this read (after the
+  // last ticket's acquire) sees it; it is issued with the partials and used last.
+  const unsigned status = *reinterpret_cast<volatile unsigned*>(&g_status);
+  const int64_t sstride = static_cast<int64_t>(p.Hq) * (128 + 2);
+  const int half_ns = (ns + 1) / 2, n_items = ng * 64;
+  const int lane = threadIdx.x & 31, half = lane >> 4;
+  for (int first = (threadIdx.x >> 5) * 16; first < n_items; first += (nthreads >> 5) * 16) {  // per warp
+    const int it = min(first + (lane & 15), n_items - 1);
+    const int h = hk * ng + (it >> 6), cp = (it & 63) * 2;
+    const float* base = p.ws + (static_cast<int64_t>(b) * p.n_split * p.Hq + h) * (128 + 2);
+    const int s_lo = half * half_ns, s_hi = min(ns, s_lo + half_ns);
+    float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f;
+    for (int s0 = s_lo; s0 < s_hi; s0 += kMergeBatch) {
+      float ms[kMergeBatch], ls[kMergeBatch];
+      float2 os[kMergeBatch];
+#pragma unroll
+      for (int u = 0; u < kMergeBatch; ++u) {  // past s_hi: the last split again, skipped below
+        const float* ps = base + min(s0 + u, s_hi - 1) * sstride;
+        ms[u] = __ldcg(ps);
+        ls[u] = __ldcg(ps + 1);
+        os[u] = __ldcg(reinterpret_cast<const float2*>(ps + 2 + cp));
+      }
+      float mb = M;
+#pragma unroll
+      for (int u = 0; u < kMergeBatch; ++u)
+        if (s0 + u < s_hi) mb = fmaxf(mb, ms[u]);
+      if (mb == -INFINITY) continue;
+      if (mb > M) {  // rescale what is summed so far to the new maximum
+        const float r = (M == -INFINITY) ? 0.f : ex2_approx(M - mb);
+        l *= r;
+        a0 *= r;
+        a1 *= r;
+        M = mb;
+      }
+#pragma unroll
+      for (int u = 0; u < kMergeBatch; ++u) {
+        const float sc = (s0 + u < s_hi && ms[u] != -INFINITY) ? ex2_approx(ms[u] - M) : 0.f;
+        l = fmaf(ls[u], sc, l);
+        a0 = fmaf(os[u].x, sc, a0);
+        a1 = fmaf(os[u].y, sc, a1);
+      }
+    }
+    // join the two halves (lane l ^ 16 holds the other one)
+    const float Mo = __shfl_xor_sync(0xffffffffu, M, 16), lo_ = __shfl_xor_sync(0xffffffffu, l, 16);
+    const float a0o = __shfl_xor_sync(0xffffffffu, a0, 16), a1o = __shfl_xor_sync(0xffffffffu, a1, 16);
+    const float Mx = fmaxf(M, Mo);
+    const float r = (M == -INFINITY) ? 0.f : ex2_approx(M - Mx), ro = (Mo == -INFINITY) ? 0.f : ex2_approx(Mo - Mx);
+    l = l * r + lo_ * ro;
+    a0 = a0 * r + a0o * ro;
+    a1 = a1 * r + a1o * ro;
+    if (half == 0 && first + lane < n_items) {
+      // a split gave up: its partials are stale, so the output is marked undefined
+      const bool bad = failed || (status & kDevErrTimeout) != 0;
+      const float nan = __int_as_float(0x7fc00000);
+      *reinterpret_cast<uint32_t*>(p.out + (static_cast<int64_t>(b) * p.Hq + h) * 128 + cp) =
+          bad ? pack_bf16x2(nan, nan) : pack_bf16x2(a0 / l, a1 / l);
+      if (cp == 0 && p.lse != nullptr)
+        p.lse[static_cast<int64_t>(b) * p.Hq + h] = bad ? nan : (Mx + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+}
 
 // warps 2-3 and 8.. correct keys; 4-7 (one TMEM lane quarter each) run the softmax
 __device__ __forceinline__ int dec_rot_index(int warp) {
@@ -188,23 +322,9 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
 
   const int hk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int ng = p.group;  // query heads of this KV head (<= GROUP; the rest of the capacity is zero rows)
-  griddep_wait();              // the query, the cache rows and the lengths may come from the previous kernel
-  griddep_launch_dependents();  // the combine step may be scheduled now; it waits for this grid to finish
-  const int L = p.seqlens[b];
-  const int c0 = split * p.chunk;
-  if (c0 >= L) return;
-  if (status_failed()) return;
-  const int c1 = min(c0 + p.chunk, L);
-  const int n_tiles = (c1 - c0 + kDecTile - 1) / kDecTile;
-  const int i = L - 1;
-  int G = 1, jb = -1;  // remote keys are j <= jb
-  if (!PLAIN) {
-    G = max(1, (L + p.w_pre - 1) / p.w_pre);
-    if (G > 1) jb = i - p.w0;
-  }
-  const int64_t row0 = static_cast<int64_t>(b) * p.cache_stride;  // token row of this entry's first key
-  // the grid covers the length; the query's correction row is in the table
-  JL_CHECK(L <= p.n_split * p.chunk && i < p.n_tab_rows && (i - i / G) < p.n_tab_rows && hk * ng + ng <= p.Hq);
+  // The next kernel in the stream may be scheduled now: it sets itself up and waits for
+  // this whole grid before it reads anything (the combine step, or the next decode).
+  griddep_launch_dependents();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -217,6 +337,8 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Setup that touches only this CTA's shared and tensor memory runs before the wait
+  // for the previous kernel, so it overlaps that kernel's tail.
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -235,23 +357,59 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     mbar_init(&bars->red_full[0], 128);
     mbar_init(&bars->red_full[1], 128);
     mbar_init(&bars->red_end, 128);
+    mbar_init(&bars->fin, 128);
     bars->abort = 0;
+    bars->last = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, Lay::kTmemCols);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  griddep_wait();  // the query, the cache rows and the lengths may come from the previous kernel
+  // One thread decides whether this CTA works (its keys exist, and no kernel has given up
+  // on a bounded wait), so that the whole CTA takes the same path.
+  if (threadIdx.x == 0) bars->last = (split * p.chunk >= p.seqlens[b]) ? 2 : status_failed() ? 1 : 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  const int L = p.seqlens[b];
+  const int c0 = split * p.chunk;
+  const int n_active = (L + p.chunk - 1) / p.chunk;  // split CTAs of (b, hk) that write partials
+  if (bars->last != 0) {
+    // Past the entry's length: nothing to do.  After a failure: skip the work, but still
+    // take the ticket so that the last CTA marks the output undefined and the counter
+    // is left clear.
+    const bool failed = bars->last == 1;
+    __syncthreads();
+    if (failed && p.counters != nullptr) {
+      if (threadIdx.x == 0) bars->last = take_ticket(p.counters + 2 * (b * p.Hkv + hk), p.epoch, n_active);
+      __syncthreads();
+      if (bars->last) merge_head_group(p, b, hk, ng, n_active, Lay::kThreads, true);
+    }
+    if (warp == 1) tmem_dealloc(tmem, Lay::kTmemCols);
+    return;
+  }
+  const int c1 = min(c0 + p.chunk, L);
+  const int n_tiles = (c1 - c0 + kDecTile - 1) / kDecTile;
+  const int i = L - 1;
+  int G = 1, jb = -1;  // remote keys are j <= jb
+  if (!PLAIN) {
+    G = max(1, (L + p.w_pre - 1) / p.w_pre);
+    if (G > 1) jb = i - p.w0;
+  }
+  const int64_t row0 = static_cast<int64_t>(b) * p.cache_stride;  // token row of this entry's first key
+  // the grid covers the length; the query's correction row is in the table
+  JL_CHECK(L <= p.n_split * p.chunk && i < p.n_tab_rows && (i - i / G) < p.n_tab_rows && hk * ng + ng <= p.Hq);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       int issued[kDecStages] = {0};
       StepDiv pdiv{};  // page and row of the tile's first key, stepped per tile (paged caches)
       if (p.block_table != nullptr) pdiv.init(c0, kDecTile, p.page_size);
@@ -413,27 +571,44 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
     // Query operand: rows 0..15 remote-corrected R(f(i) - i) q~, rows 16..31 q~; zero padding.
+    // Thread = (head g, channels c..c+7 and c+64..c+71): all of its loads (two 16-byte
+    // query words, and for G > 1 the correction row's cos/sin) go out before any is used.
     {
-      const int nq = i - i / G;
-      for (int e = tid; e < kDecQRows * 64; e += 128) {
-        const int row = e >> 6, c = e & 63;
-        const int g = row & 15;
-        float lo = 0.f, hi = 0.f;
-        if (g < ng) {
-          const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * ng + g) * 128;
-          lo = __bfloat162float(qp[c]);
-          hi = __bfloat162float(qp[c + 64]);
-          if (row < 16 && G > 1 && !PLAIN) {
-            const float cs = p.cos_tab[static_cast<int64_t>(nq) * 64 + c];
-            const float sn = p.sin_tab[static_cast<int64_t>(nq) * 64 + c];
-            const float a = lo, bb = hi;
-            lo = a * cs + bb * sn;
-            hi = bb * cs - a * sn;
-          }
+      const int g = tid >> 3, c = (tid & 7) * 8;
+      uint4 qlo = make_uint4(0, 0, 0, 0), qhi = qlo;
+      float4 c0v = make_float4(0.f, 0.f, 0.f, 0.f), c1v = c0v, s0v = c0v, s1v = c0v;
+      if (g < ng) {
+        const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.Hq + hk * ng + g) * 128 + c;
+        qlo = *reinterpret_cast<const uint4*>(qp);
+        qhi = *reinterpret_cast<const uint4*>(qp + 64);
+        if (G > 1 && !PLAIN) {
+          const int64_t nq = i - i / G;  // correction index of the query
+          const float4* cp = reinterpret_cast<const float4*>(p.cos_tab + nq * 64 + c);
+          const float4* sp = reinterpret_cast<const float4*>(p.sin_tab + nq * 64 + c);
+          c0v = cp[0];
+          c1v = cp[1];
+          s0v = sp[0];
+          s1v = sp[1];
         }
-        *reinterpret_cast<__nv_bfloat16*>(sQ + swz_off(row, c, kDecQRows * 128)) = __float2bfloat16_rn(lo);
-        *reinterpret_cast<__nv_bfloat16*>(sQ + swz_off(row, c + 64, kDecQRows * 128)) = __float2bfloat16_rn(hi);
       }
+      const uint32_t lw[4] = {qlo.x, qlo.y, qlo.z, qlo.w}, hw[4] = {qhi.x, qhi.y, qhi.z, qhi.w};
+      uint32_t rlo[4] = {lw[0], lw[1], lw[2], lw[3]}, rhi[4] = {hw[0], hw[1], hw[2], hw[3]};
+      if (G > 1 && !PLAIN) {
+        const float cs[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+        const float sn[8] = {s0v.x, s0v.y, s0v.z, s0v.w, s1v.x, s1v.y, s1v.z, s1v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // (lo, hi) -> (lo c + hi s, hi c - lo s), channels 2e, 2e + 1
+          const float2 a = unpack_bf16x2(lw[e]), bb = unpack_bf16x2(hw[e]);
+          rlo[e] = pack_bf16x2(a.x * cs[2 * e] + bb.x * sn[2 * e], a.y * cs[2 * e + 1] + bb.y * sn[2 * e + 1]);
+          rhi[e] = pack_bf16x2(bb.x * cs[2 * e] - a.x * sn[2 * e], bb.y * cs[2 * e + 1] - a.y * sn[2 * e + 1]);
+        }
+      }
+      // 8 channels = one 16-byte chunk of a swizzled row (c is a multiple of 8)
+      *reinterpret_cast<uint4*>(sQ + swz_off(g, c, kDecQRows * 128)) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
+      *reinterpret_cast<uint4*>(sQ + swz_off(g, c + 64, kDecQRows * 128)) =
+          make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
+      *reinterpret_cast<uint4*>(sQ + swz_off(16 + g, c, kDecQRows * 128)) = qlo;
+      *reinterpret_cast<uint4*>(sQ + swz_off(16 + g, c + 64, kDecQRows * 128)) = qhi;
       // both P buffers start at zero (rows >= GROUP are never written)
       for (int e = tid; e < 2 * kDecHeads * 256 / 16; e += 128)
         reinterpret_cast<uint4*>(sP)[e] = make_uint4(0, 0, 0, 0);
@@ -535,6 +710,15 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
       }
       }
     }
+    if (p.counters != nullptr) {
+      // Every softmax thread, on every path (an aborted CTA takes a ticket too, so the
+      // count completes): the arrival orders its partial stores before the ticket.
+      mbar_arrive(&bars->fin);
+      if (tid == 0) {
+        mbar_wait_bounded(&bars->fin, 0);
+        bars->last = take_ticket(p.counters + 2 * (b * p.Hkv + hk), p.epoch, n_active);
+      }
+    }
   }
 
   tc_fence_before();
@@ -543,6 +727,8 @@ __global__ void __launch_bounds__(DecTcLayout<GROUP>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
   }
+  if (bars->last)  // uniform; set only with p.counters (the ticket acquired the other partials)
+    merge_head_group(p, b, hk, ng, n_active, Lay::kThreads, false);
 }
 
 }  // namespace jl

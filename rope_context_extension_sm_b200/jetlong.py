@@ -36,6 +36,7 @@ SIGNATURES = {
     "jl_group_size": (_i64, [_i64, _i64]),
     "jl_sync_status": (ctypes.c_int, [_vp]),
     "jl_debug_bounds_enabled": (ctypes.c_int, []),
+    "jl_decode_single_launch_enabled": (ctypes.c_int, []),
     "jl_rope_tables": (ctypes.c_int, [_vp, _vp, _i64, _i32, _f64, _vp]),
     "jl_bifocal_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
                                           _vp, _vp, _i64, _f32, _vp, _vp, _vp]),

@@ -101,12 +101,13 @@ def test_decode_workspace_size(jlmod):
 def test_decode_workspace_covers_a_one_wave_split_for_every_kv_head_count(jlmod, B, Hq, L):
     # The tensor-core decode runs at most one wave of 148 CTAs (B x Hkv x splits), each
     # split a whole number of 128-key tiles; the size query does not know Hkv, so it has
-    # to cover the largest split any Hkv allowed by Hq can produce.
+    # to cover the largest split any Hkv allowed by Hq can produce, plus two 8-byte merge
+    # counter words per (entry, KV head) after the partials.
     n = jlmod.jl_bifocal_decode_workspace_size(B, Hq, 128, L)
     tiles = -(-L // 128)
     for hkv in [h for h in range(1, Hq + 1) if Hq % h == 0 and Hq // h <= 16]:
         worst_split = min(tiles, max(1, 148 // (hkv * B)))
-        assert n >= B * worst_split * Hq * (128 + 2) * 4, hkv
+        assert n >= B * worst_split * Hq * (128 + 2) * 4 + B * hkv * 16, hkv
 
 
 def test_prefill_and_cache_rejects_a_short_cache_without_launching(jlmod):

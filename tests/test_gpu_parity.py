@@ -363,6 +363,55 @@ def test_decode_replayed_from_a_cuda_graph_follows_the_device_lengths(jl):
     del g
 
 
+def test_decode_workspace_of_random_bytes(jl):
+    """The last CTA of each (entry, KV head) merges the split partials; it is found through
+    counter words in the workspace that carry a per-call tag.  A workspace full of random
+    bytes (counter words with arbitrary tags and counts) must give the oracle's result, and
+    so must a second call on the same workspace and a call after the words were zeroed."""
+    cfg = SMALL_DECODE
+    max_len, L = 1024, 1000  # 8 splits of one 128-key tile per KV head
+    k_cache, v = _decode_setup(cfg, max_len)
+    kd, vd = k_cache.cuda(), v.cuda()
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    q_t = _query_tilde(cfg, I.decode_queries(cfg, 1)[0, 0], L)
+    qd = q_t[None].cuda().contiguous()
+    sl = torch.tensor([L], dtype=torch.int32, device="cuda")
+    n = jl.jl_bifocal_decode_workspace_size(1, cfg.n_q_heads, cfg.head_dim, max_len)
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, generator=gen).cuda()
+    ro, rl = _decode_oracle(cfg, q_t, k_cache[0], v[0], L)
+    first = None
+    for call in ("random", "again", "zeroed"):
+        if call == "zeroed":
+            ws.zero_()
+        out, lse = jl.jl_bifocal_decode(qd, kd, vd, sl, max_len, cfg.w0, cfg.w_pretrained, cos, sin, workspace=ws)
+        jl.jl_sync_status()
+        got = (out.float().cpu().numpy()[0], lse.cpu().numpy()[0])
+        _check(got[0], got[1], ro, rl, f"decode, workspace {call}")
+        if first is None:
+            first = got
+        else:
+            assert np.array_equal(first[0], got[0]) and np.array_equal(first[1], got[1]), call
+
+
+def test_batched_decode_more_ctas_than_one_wave(jl):
+    """10 entries x 8 KV heads x 2 splits = 160 CTAs on 148 SMs: the split CTAs of one (entry,
+    KV head) can run in different waves, and entries no longer than the split size (16384
+    keys) have one active split, which is then its own last CTA.  Random rows stand for the
+    base-rotated keys (the decode only reads the cache)."""
+    cfg = I.DecodeConfig("wave", (), 32, 8, 128, 1024, 4096, 1e6)
+    lens = [20000, 19000, 300, 16385, 129, 20000, 8000, 16384, 1, 12345]
+    max_len = 20000
+    k_cache, v = I.decode_raw_inputs(cfg, max_len, len(lens))
+    qs = I.decode_queries(cfg, 1, batch=len(lens))[0]
+    q_t = torch.stack([_query_tilde(cfg, qs[b], lens[b]) for b in range(len(lens))])
+    cos, sin = _tables(jl, max_len, cfg.head_dim, cfg.rope_base)
+    out, lse = _run_decode(jl, cfg, q_t, k_cache.cuda(), v.cuda(), lens, max_len, cos, sin)
+    for b, L in enumerate(lens):
+        ro, rl = _decode_oracle(cfg, q_t[b], k_cache[b], v[b], L)
+        _check(out[b], lse[b], ro, rl, f"multi-wave decode b={b} L={L} G={O.group_size(L, 4096)}")
+
+
 def test_batched_decode_each_sequence_its_own_G(jl):
     cfg = SMALL_DECODE
     max_len, lens = 1024, [1024, 250, 513, 7]
