@@ -203,22 +203,25 @@ def _measure_other_configs(jl, dev, sustained, hbm, _time, _time_graph):
     cos, sin = jl.jl_rope_tables(L, cfg.head_dim, cfg.rope_base, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty((cfg.n_q_heads, L), dtype=torch.float32, device=dev)
+    kws = torch.empty(jl.jl_bifocal_prefill_workspace_size(L, cfg.n_kv_heads, cfg.head_dim), dtype=torch.uint8,
+                      device=dev)
     flops = cfg.useful_flops()
     sweep = {}
     for _ in range(10):  # ~0.2 s of the same work first, so every point runs at the steady-state clock
-        jl.jl_bifocal_prefill(q, k, v, cu, L, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+        jl.jl_bifocal_prefill(q, k, v, cu, L, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse, workspace=kws)
     for w0 in I.W0_SWEEP:
-        fn = lambda w0=w0: jl.jl_bifocal_prefill(q, k, v, cu, L, w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+        fn = lambda w0=w0: jl.jl_bifocal_prefill(q, k, v, cu, L, w0, cfg.w_pretrained, cos, sin, out=out, lse=lse,
+                                                 workspace=kws)
         fn()
         ms = _time(fn, 5)
         sweep[str(w0)] = {"ms": round(ms, 3), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                           "frac_of_bf16_peak_measured_sustained": round(flops / (ms * 1e-3) / 1e12 / sustained, 4)}
-    pl = lambda: jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse)
+    pl = lambda: jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse, workspace=kws)
     pl()
     ms = _time(pl, 5)
     res["qwen3_1p7b_L65536_G2"] = {"w0_sweep": sweep, "plain_ms": round(ms, 3),
                                    "plain_useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
-    del q, k, v, out, lse, cos, sin
+    del q, k, v, out, lse, cos, sin, kws
 
     cfg = I.VARLEN
     q, k, v, cu = [t.to(dev) for t in I.prefill_inputs(cfg)]
@@ -226,8 +229,11 @@ def _measure_other_configs(jl, dev, sustained, hbm, _time, _time_graph):
     cos, sin = jl.jl_rope_tables(mx, cfg.head_dim, cfg.rope_base, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty((cfg.n_q_heads, q.shape[0]), dtype=torch.float32, device=dev)
+    kws = torch.empty(jl.jl_bifocal_prefill_workspace_size(q.shape[0], cfg.n_kv_heads, cfg.head_dim),
+                      dtype=torch.uint8, device=dev)
     flops = cfg.useful_flops()
-    fn = lambda: jl.jl_bifocal_prefill(q, k, v, cu, mx, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse)
+    fn = lambda: jl.jl_bifocal_prefill(q, k, v, cu, mx, cfg.w0, cfg.w_pretrained, cos, sin, out=out, lse=lse,
+                                       workspace=kws)
     fn()
     ms = _time(fn, 3)
     res["varlen_8seq"] = {"seqlens": list(cfg.seqlens), "ms": round(ms, 3),
@@ -465,10 +471,14 @@ def run_ours(args, world, rank, local):
     dlse = torch.empty((1, DECODE.n_q_heads), dtype=torch.float32, device=dev)
     dws = torch.empty(jl.jl_bifocal_decode_workspace_size(1, DECODE.n_q_heads, DECODE.head_dim, DECODE_L),
                       dtype=torch.uint8, device=dev)
+    # the prefill's rotated keys (base and remote rows), written by its first kernel each call
+    kws = torch.empty(jl.jl_bifocal_prefill_workspace_size(L, PREFILL.n_kv_heads, PREFILL.head_dim),
+                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def prefill():
-        jl.jl_bifocal_prefill(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin, out=out, lse=lse)
+        jl.jl_bifocal_prefill(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin, out=out, lse=lse,
+                              workspace=kws)
 
     def decode():
         jl.jl_bifocal_decode(dq, dk, dv, dsl, DECODE_L, DECODE.w0, DECODE.w_pretrained, cos, sin, out=dout,
@@ -512,7 +522,7 @@ def run_ours(args, world, rank, local):
 
     # ---- plain comparators, same run ----
     def plain_prefill():
-        jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse)
+        jl.jl_plain_prefill(q, k, v, cu, L, cos, sin, out=out, lse=lse, workspace=kws)
 
     def plain_decode():
         jl.jl_plain_decode(dq, dk, dv, dsl, DECODE_L, cos, sin, out=dout, lse=dlse, workspace=dws)
@@ -631,7 +641,7 @@ def run_ours(args, world, rank, local):
         if s_ >= 2:
             stream.wait_event(ev_out[s_ - 2])  # step s-2's results have left this buffer
         jl.jl_bifocal_prefill(d["q"], d["k"], d["v"], cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin,
-                              out=d["out"], lse=d["lse"])
+                              out=d["out"], lse=d["lse"], workspace=kws)
         jl.jl_bifocal_decode(d["dq"], dk, dv, dsl, DECODE_L, DECODE.w0, DECODE.w_pretrained, cos, sin,
                              out=d["dout"], lse=dlse, workspace=dws)
         ev_done[s_].record(stream)
@@ -710,6 +720,8 @@ def run_ours(args, world, rank, local):
             "frac": round(prefill_tflops / sustained, 4),
             "traffic": _traffic("prefill", PREFILL_SRC),
             "tensor_pipe_active": _profiled("prefill", PREFILL_SRC, "tensor_pipe_active_pct"),
+            # the timed call is the whole jl_bifocal_prefill: the keys' rotation kernel, then this kernel
+            "duration_includes": "jl_key_rotate_kernel",
             "algorithmic_bytes_per_launch": int(sum(t.numel() * t.element_size() for t in (q, k, v, out, lse))),
         },
         "e2e": {
@@ -719,7 +731,8 @@ def run_ours(args, world, rank, local):
             "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h),
         },
-        "gpu_launches": 3 * K,  # per step: the prefill kernel, the decode split kernel and its merge
+        # per step: the key rotation and the prefill kernel, the decode split kernel and its merge
+        "gpu_launches": 4 * K,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_cpu_baseline:

@@ -160,14 +160,29 @@ jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const i
  *   out         bf16 [total_tokens][Hq][head_dim]
  *   lse         fp32 [Hq][total_tokens], natural-log log-sum-exp of the scaled
  *               routed scores of each row; may be NULL.
+ *   workspace   NULL, or device scratch of at least
+ *               jl_bifocal_prefill_workspace_size(total_tokens, Hkv, head_dim)
+ *               bytes, 16-byte aligned, owned by the caller; its contents on
+ *               entry do not matter.  With a workspace the keys are rotated once,
+ *               before the attention kernel: the workspace receives R(j) k_j and,
+ *               for sequences with G > 1, R(f(j)) k_j, and the kernel reads those
+ *               for its local and remote visits.  Without one (NULL, 0) the
+ *               kernel rotates each key tile on every visit (no global scratch).
+ *               Both give the routed scores of the method; they may differ in the
+ *               last bf16 bit of a rotated key (table row against a rotation
+ *               recurrence), well inside the parity tolerance.
  * Supported: head_dim in {64, 128}; Hq % Hkv == 0; batch >= 0 (0 is a no-op).
- * No workspace; the kernel keeps everything in shared and tensor memory.
  */
 jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
                              int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv,
                              int32_t head_dim, int32_t w0, int32_t w_pretrained, const float* cos_tab,
                              const float* sin_tab, int64_t n_tab_rows, float softmax_scale, void* out, float* lse,
-                             jl_stream_t stream);
+                             void* workspace, size_t workspace_bytes, jl_stream_t stream);
+
+/* Bytes of the jl_bifocal_prefill / jl_plain_prefill workspace: two rotated key rows
+ * (base and remote) per token and KV head, 2 * total_tokens * Hkv * head_dim * 2.
+ * 0 for non-positive sizes. */
+size_t jl_bifocal_prefill_workspace_size(int64_t total_tokens, int32_t Hkv, int32_t head_dim);
 
 /*
  * jl_bifocal_prefill that also writes the base-RoPE KV cache the decode reads
@@ -241,11 +256,12 @@ jl_status jl_bifocal_prefill_three_pass(const void* q, const void* k, const void
 size_t jl_bifocal_prefill_three_pass_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim);
 
 /* Plain causal RoPE prefill (every causal pair LOCAL), built from the same
- * kernel; the comparator for bifocal prefill.  Same conventions. */
+ * kernel; the comparator for bifocal prefill.  Same conventions, workspace
+ * included (only its base rows are written). */
 jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                            int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                            const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,
-                           void* out, float* lse, jl_stream_t stream);
+                           void* out, float* lse, void* workspace, size_t workspace_bytes, jl_stream_t stream);
 
 /*
  * Single-query bifocal decode with the on-the-fly correction rotation

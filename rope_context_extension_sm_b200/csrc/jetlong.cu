@@ -140,9 +140,10 @@ jl_status launch_prefill(const void* q, const void* k, const void* v, const jl::
   CUtensorMap tq, tk, tv;
   jl_status s;
   if ((s = make_map(&tq, q, prm.total_tokens, prm.Hq, D)) != JL_OK) return s;
-  // keys/values: the packed prompt, or (chunked prefill) the base-RoPE caches
+  // keys/values: the packed prompt, or (chunked prefill) the base-RoPE caches; pre-rotated
+  // keys hold a base and a remote row per token
   const int64_t kv_rows = prm.cached ? static_cast<int64_t>(prm.batch) * prm.cache_stride : prm.total_tokens;
-  if ((s = make_map(&tk, k, kv_rows, prm.Hkv, D)) != JL_OK) return s;
+  if ((s = make_map(&tk, k, prm.krot ? 2 * prm.total_tokens : kv_rows, prm.Hkv, D)) != JL_OK) return s;
   if ((s = make_map(&tv, v, kv_rows, prm.Hkv, D)) != JL_OK) return s;
   auto kern = jl::jl_prefill_kernel<D, NQT>;
   const KernelAttr attr = kernel_attr(reinterpret_cast<const void*>(kern), Lay::kAlloc);
@@ -223,7 +224,7 @@ jl_status launch_prefill_db(const void* q, const void* k, const void* v, jl::Pre
   jl_status s;
   if ((s = make_map(&tq, q, prm.total_tokens, prm.Hq, D)) != JL_OK) return s;
   const int64_t kv_rows = prm.cached ? static_cast<int64_t>(prm.batch) * prm.cache_stride : prm.total_tokens;
-  if ((s = make_map(&tk, k, kv_rows, prm.Hkv, D)) != JL_OK) return s;
+  if ((s = make_map(&tk, k, prm.krot ? 2 * prm.total_tokens : kv_rows, prm.Hkv, D)) != JL_OK) return s;
   if ((s = make_map(&tv, v, kv_rows, prm.Hkv, D)) != JL_OK) return s;
   auto kern = jl::jl_prefill_db_kernel<D>;
   const KernelAttr attr = kernel_attr(reinterpret_cast<const void*>(kern), Lay::kAlloc);
@@ -260,17 +261,53 @@ jl_status launch_prefill_any(const void* q, const void* k, const void* v, const 
   return pair ? launch_prefill<64, 2>(q, k, v, prm, st) : launch_prefill<64, 1>(q, k, v, prm, st);
 }
 
+// Bytes of the pre-rotated keys: a base row R(j) k and a remote row R(f(j)) k per
+// token and KV head.
+size_t key_rot_bytes(int64_t total_tokens, int32_t Hkv, int32_t head_dim) {
+  if (total_tokens <= 0 || Hkv <= 0 || head_dim <= 0) return 0;
+  return 2 * static_cast<size_t>(total_tokens) * Hkv * head_dim * sizeof(__nv_bfloat16);
+}
+
+// With a workspace, the keys are rotated once into it (jl_key_rotate_kernel) and the
+// prefill kernel reads them as they are; without one, its rotation warps rotate every
+// key tile on every visit.
 jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                          int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                          int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
-                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, cudaStream_t st) {
+                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, cudaStream_t st) {
   jl::PrefillParams prm;
   bool empty;
   jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
                                w_pretrained, plain, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
                                &empty);
   if (s != JL_OK || empty) return s;
-  return launch_prefill_any(q, k, v, prm, head_dim, st);
+  if (workspace == nullptr) return launch_prefill_any(q, k, v, prm, head_dim, st);
+  const size_t need = key_rot_bytes(total_tokens, Hkv, head_dim);
+  if (workspace_bytes < need)
+    return fail(JL_ERR_INVALID, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(JL_ERR_INVALID, "the workspace must be 16-byte aligned");
+  if (total_tokens >= (int64_t(1) << 30))  // the remote rows sit total_tokens rows on, as int32 TMA coordinates
+    return fail(JL_ERR_UNSUPPORTED, "a key workspace needs total_tokens < 2^30 (got %lld)", (long long)total_tokens);
+  jl::AppendParams ap{};
+  ap.k = static_cast<const __nv_bfloat16*>(k);
+  ap.lens = cu_seqlens;
+  ap.cos_tab = cos_tab;
+  ap.sin_tab = sin_tab;
+  ap.k_cache = static_cast<__nv_bfloat16*>(workspace);
+  ap.total_tokens = total_tokens;
+  ap.n_tab_rows = n_tab_rows;
+  ap.batch = batch;
+  ap.Hkv = Hkv;
+  ap.w_pre = plain ? 0x7fffffff : w_pretrained;  // plain: every pair is local, no remote rows
+  const int64_t warps = (total_tokens * Hkv + jl::kFillRowsPerWarp - 1) / jl::kFillRowsPerWarp;
+  const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+  if (head_dim == 128) jl::jl_key_rotate_kernel<128><<<blocks, 256, 0, st>>>(ap);
+  else jl::jl_key_rotate_kernel<64><<<blocks, 256, 0, st>>>(ap);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
+  prm.krot = 1;
+  return launch_prefill_any(q, workspace, v, prm, head_dim, st);
 }
 
 size_t three_pass_ws_bytes(int64_t total_tokens, int32_t Hq, int32_t head_dim) {
@@ -654,10 +691,15 @@ jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t 
 jl_status jl_bifocal_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                              int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                              int32_t w0, int32_t w_pretrained, const float* cos_tab, const float* sin_tab,
-                             int64_t n_tab_rows, float softmax_scale, void* out, float* lse, jl_stream_t stream) {
+                             int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, jl_stream_t stream) {
   return prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0, w_pretrained,
-                        0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse,
+                        0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, workspace, workspace_bytes,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t jl_bifocal_prefill_workspace_size(int64_t total_tokens, int32_t Hkv, int32_t head_dim) {
+  return key_rot_bytes(total_tokens, Hkv, head_dim);
 }
 
 jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
@@ -694,9 +736,10 @@ jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void*
 jl_status jl_plain_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                            int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                            const float* cos_tab, const float* sin_tab, int64_t n_tab_rows, float softmax_scale,
-                           void* out, float* lse, jl_stream_t stream) {
+                           void* out, float* lse, void* workspace, size_t workspace_bytes, jl_stream_t stream) {
   return prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, 0, 1, 1, cos_tab,
-                        sin_tab, n_tab_rows, softmax_scale, out, lse, reinterpret_cast<cudaStream_t>(stream));
+                        sin_tab, n_tab_rows, softmax_scale, out, lse, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 jl_status jl_kv_cache_fill(const void* k, const void* v, const int32_t* cu_seqlens, const int32_t* past_lens,

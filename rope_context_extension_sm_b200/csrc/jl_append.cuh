@@ -7,6 +7,7 @@
 //
 // jl_kv_fill_kernel     prompt tokens (packed varlen) -> cache entries
 // jl_decode_append_kernel  one new token per entry: q~ = R(i) q, cache[i] = R(i) k, v
+// jl_key_rotate_kernel  prompt keys -> the prefill's pre-rotated key rows (base and remote)
 // The fill kernel gives each warp four (token, head) rows, the append kernel one;
 // lanes own rotate-half pairs (c, c + D/2) and every access is a coalesced row read
 // or write.
@@ -35,6 +36,7 @@ struct AppendParams {
   int32_t batch, Hq, Hkv;
   const int32_t* block_table;  // paged caches (NULL: contiguous [batch][cache_stride])
   int32_t page_size, max_pages, num_pages;
+  int32_t w_pre;               // key rotation: w_pretrained, for G per sequence
 };
 
 // Cache row of entry b's position pos (already checked against cache_stride):
@@ -154,6 +156,104 @@ __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
       p.k_cache[dst[r] + lane] = __float2bfloat16_rn(ka[r] * cs[r] - kb[r] * sn[r]);
       p.k_cache[dst[r] + HALF + lane] = __float2bfloat16_rn(kb[r] * cs[r] + ka[r] * sn[r]);
       *reinterpret_cast<uint32_t*>(p.v_cache + dst[r] + 2 * lane) = vw[r];
+    }
+  }
+}
+
+// Keys for the bifocal prefill, rotated once before it instead of on every visit
+// inside it ("Jet-Long", Methodology section 1: local pairs use the base positions,
+// remote pairs the grouped positions f(x) = floor(x / G)).  Token t of sequence b sits
+// at position j = t - cu_seqlens[b]; with G = max(1, ceil(L_b / w_pretrained)):
+//   k_out[t]     = R(j) k_t          (local visits)
+//   k_out[T + t] = R(floor(j / G)) k_t  (remote visits; not written for G = 1, whose
+//                                       pairs are all local)
+// Same lane layout and load batching as jl_kv_fill_kernel; p.k_cache is the output.
+template <int D>
+__global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p) {
+  constexpr int R = kFillRowsPerWarp;
+  constexpr int HALF = D / 2;
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32 * R;
+  const int lane = threadIdx.x & 31;
+  const int64_t n_rows = p.total_tokens * p.Hkv;
+  const int64_t remote_off = p.total_tokens * p.Hkv * D;  // element offset of the remote rows
+  int64_t src[R], pos[R], fpos[R];
+  bool live[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {  // locate each row: its sequence, position and G
+    const int64_t row = row0 + r;
+    live[r] = row < n_rows;
+    src[r] = pos[r] = 0;
+    fpos[r] = -1;
+    if (!live[r]) continue;
+    const int64_t t = row / p.Hkv;
+    const int h = static_cast<int>(row % p.Hkv);
+    int lo = 0, hi = p.batch - 1;  // sequence holding token t: last b with cu[b] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.lens[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int L = p.lens[b + 1] - p.lens[b];
+    const int G = max(1, (L + p.w_pre - 1) / p.w_pre);
+    pos[r] = t - p.lens[b];
+    if (pos[r] < 0 || pos[r] >= p.n_tab_rows) {  // the host checks max_seqlen <= n_tab_rows
+      if (lane == 0) atomicOr(&g_status, kDevErrBounds);
+      live[r] = false;
+      continue;
+    }
+    if (G > 1) fpos[r] = pos[r] / G;
+    src[r] = (t * p.Hkv + h) * D;
+  }
+  if constexpr (D == 128) {
+    uint32_t ka[R], kb[R];
+    float2 cs[R], sn[R], cf[R], sf[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      ka[r] = *reinterpret_cast<const uint32_t*>(p.k + src[r] + 2 * lane);
+      kb[r] = *reinterpret_cast<const uint32_t*>(p.k + src[r] + HALF + 2 * lane);
+      cs[r] = *reinterpret_cast<const float2*>(p.cos_tab + pos[r] * HALF + 2 * lane);
+      sn[r] = *reinterpret_cast<const float2*>(p.sin_tab + pos[r] * HALF + 2 * lane);
+      const int64_t fr = fpos[r] >= 0 ? fpos[r] : 0;
+      cf[r] = *reinterpret_cast<const float2*>(p.cos_tab + fr * HALF + 2 * lane);
+      sf[r] = *reinterpret_cast<const float2*>(p.sin_tab + fr * HALF + 2 * lane);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      const float2 a = unpack_bf16x2(ka[r]);
+      const float2 bb = unpack_bf16x2(kb[r]);
+      *reinterpret_cast<uint32_t*>(p.k_cache + src[r] + 2 * lane) =
+          pack_bf16x2(a.x * cs[r].x - bb.x * sn[r].x, a.y * cs[r].y - bb.y * sn[r].y);
+      *reinterpret_cast<uint32_t*>(p.k_cache + src[r] + HALF + 2 * lane) =
+          pack_bf16x2(bb.x * cs[r].x + a.x * sn[r].x, bb.y * cs[r].y + a.y * sn[r].y);
+      if (fpos[r] < 0) continue;
+      *reinterpret_cast<uint32_t*>(p.k_cache + remote_off + src[r] + 2 * lane) =
+          pack_bf16x2(a.x * cf[r].x - bb.x * sf[r].x, a.y * cf[r].y - bb.y * sf[r].y);
+      *reinterpret_cast<uint32_t*>(p.k_cache + remote_off + src[r] + HALF + 2 * lane) =
+          pack_bf16x2(bb.x * cf[r].x + a.x * sf[r].x, bb.y * cf[r].y + a.y * sf[r].y);
+    }
+  } else {
+    float ka[R], kb[R], cs[R], sn[R], cf[R], sf[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      ka[r] = __bfloat162float(p.k[src[r] + lane]);
+      kb[r] = __bfloat162float(p.k[src[r] + HALF + lane]);
+      cs[r] = p.cos_tab[pos[r] * HALF + lane];
+      sn[r] = p.sin_tab[pos[r] * HALF + lane];
+      const int64_t fr = fpos[r] >= 0 ? fpos[r] : 0;
+      cf[r] = p.cos_tab[fr * HALF + lane];
+      sf[r] = p.sin_tab[fr * HALF + lane];
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!live[r]) continue;
+      p.k_cache[src[r] + lane] = __float2bfloat16_rn(ka[r] * cs[r] - kb[r] * sn[r]);
+      p.k_cache[src[r] + HALF + lane] = __float2bfloat16_rn(kb[r] * cs[r] + ka[r] * sn[r]);
+      if (fpos[r] < 0) continue;
+      p.k_cache[remote_off + src[r] + lane] = __float2bfloat16_rn(ka[r] * cf[r] - kb[r] * sf[r]);
+      p.k_cache[remote_off + src[r] + HALF + lane] = __float2bfloat16_rn(kb[r] * cf[r] + ka[r] * sf[r]);
     }
   }
 }

@@ -84,6 +84,9 @@ struct PrefillParams {
   int32_t plain;
   int32_t mode;          // 0: fused bifocal / plain; 1: pass 1 alone; 3: pass 3 alone (see TileSchedule)
   int32_t cached;        // keys/values come from a base-RoPE cache (chunked prefill)
+  // Keys arrive rotated (jl_key_rotate_kernel): rows [0, T) of the K map hold R(j) k_j for
+  // local visits, rows [T, 2T) R(f(j)) k_j for remote visits; no K rotation in the kernel.
+  int32_t krot;
   const float* cos_rem;  // frequency-interpolation variant: remote pairs rotate by these
   const float* sin_rem;  // rows at their raw positions (cos/sin(p theta_c lambda_c)); NULL = aliasing
   int64_t n_rem_rows;
@@ -626,10 +629,12 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
                  key0 + min(kBN - 1, L - 1 - sc.kt(n) * kBN) <
                      (p.cached ? static_cast<int64_t>(b) * p.cache_stride + (L < p.cache_stride ? L : p.cache_stride)
                                : static_cast<int64_t>(seq0) + n_rows));
+        // pre-rotated keys: a remote visit reads the R(f(j)) k rows, T rows on
+        const int krow = key0 + ((p.krot && sc.remote(n)) ? static_cast<int>(p.total_tokens) : 0);
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d(sK + s * Lay::kTileBytes + bx * Lay::kBoxBytes, &tm_k, &bars->k_full[s], bx * 64, hkv, key0);
+          tma_load_3d(sK + s * Lay::kTileBytes + bx * Lay::kBoxBytes, &tm_k, &bars->k_full[s], bx * 64, hkv, krow);
         if (u > 0 && !mbar_wait(&bars->v_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->v_full[s], kTileTx);
         for (int bx = 0; bx < NBOX; ++bx)
@@ -760,7 +765,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       return p.cached ? pos - kdiv.q : kdiv.q;  // cached: correction index n_j = j - f(j)
     };
     RotFactor<D> fk_next;
-    load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
+    if (!p.krot) load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
     const bool write_cache = p.k_cache_out != nullptr && slot == 0 && p.mode == 0 && !p.cached;
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
@@ -782,7 +787,7 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
         if (lane == 0) mbar_arrive(&bars->q_ready);
       }
       const RotFactor<D> fk = fk_next;
-      if (n + 1 < sc.n_virt)  // prefetch a tile ahead
+      if (n + 1 < sc.n_virt && !p.krot)  // prefetch a tile ahead
         load_factor<D>(fk_next, p, key_anchor(n + 1), lane, interp && sc.remote(n + 1));
       const int s = n % kStages;
       {  // table rows of this slice's valid keys: base R(j), remote R(j / G) (< w_pretrained), or the
@@ -797,7 +802,9 @@ __global__ void __launch_bounds__(PrefillLayout<D, NQT>::kThreads, 1)
       JL_TRACE_AT(n, 5 + 3 * rw);
       if (!mbar_wait(&bars->k_full[s], (n / kStages) & 1, abort)) break;
       JL_TRACE_AT(n, 6 + 3 * rw);
-      if (!p.cached) {
+      if (p.krot) {
+        // the keys arrived rotated for this visit's kind
+      } else if (!p.cached) {
         rotate_slice_any<D>(sK + s * Lay::kTileBytes, rw, sc.kt(n) * kBN, g, fk, stp, lane);
         // The query block's own key tile, visited as local, now holds R(j) k_j: the first
         // head slot of the KV group writes it (and the raw V rows) to the cache before the
@@ -1225,10 +1232,12 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
                  key0 + min(kBN - 1, L - 1 - sc.kt(n) * kBN) <
                      (p.cached ? static_cast<int64_t>(b) * p.cache_stride + (L < p.cache_stride ? L : p.cache_stride)
                                : static_cast<int64_t>(seq0) + n_rows));
+        // pre-rotated keys: a remote visit reads the R(f(j)) k rows, T rows on
+        const int krow = key0 + ((p.krot && sc.remote(n)) ? static_cast<int>(p.total_tokens) : 0);
         if (u > 0 && !mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[s], kTileTx);
         for (int bx = 0; bx < NBOX; ++bx)
-          tma_load_3d(sK + s * Lay::kTileBytes + bx * Lay::kBoxBytes, &tm_k, &bars->k_full[s], bx * 64, hkv, key0);
+          tma_load_3d(sK + s * Lay::kTileBytes + bx * Lay::kBoxBytes, &tm_k, &bars->k_full[s], bx * 64, hkv, krow);
         issued[s] = static_cast<int>(u) + 1;
       }
       if (issued_q > 0) mbar_wait_bounded(&bars->q_full, (issued_q - 1) & 1);
@@ -1342,7 +1351,7 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
     };
     RotFactor8 st8, fk8_next;
     int cnt_next = 0;
-    anchor8(fk8_next, key_row(0, cnt_next), interp && sc.remote(0));
+    if (!p.krot) anchor8(fk8_next, key_row(0, cnt_next), interp && sc.remote(0));
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
       const bool rem_tab = interp && remote;
@@ -1365,7 +1374,7 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
       }
       const RotFactor8 fk8 = fk8_next;
       const int cnt_k = cnt_next;
-      if (n + 1 < sc.n_virt) anchor8(fk8_next, key_row(n + 1, cnt_next), interp && sc.remote(n + 1));
+      if (n + 1 < sc.n_virt && !p.krot) anchor8(fk8_next, key_row(n + 1, cnt_next), interp && sc.remote(n + 1));
       const int s = n % Lay::kKStages;
       {
         const int first = sc.kt(n) * kBN + RR * rw, last = min(first + RR - 1, L - 1);
@@ -1376,7 +1385,7 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
       if (!mbar_wait(&bars->k_full[s], (n / Lay::kKStages) & 1, abort)) break;
       if (rw < 4) JL_TRACE_AT(n, 6 + 3 * rw);
       uint8_t* tile = sK + s * Lay::kTileBytes;
-      rotate_slice_v128_any(tile, rw, sc.kt(n) * kBN, cnt_k, g, fk8, st8, lane);
+      if (!p.krot) rotate_slice_v128_any(tile, rw, sc.kt(n) * kBN, cnt_k, g, fk8, st8, lane);
       if (write_cache && !remote && sc.kt(n) == qt) {
         __syncwarp();
         write_cache_slice<D, RR>(tile, rw, p, b, qt * kBN, n_rows - qt * kBN, q_tok0, hkv, lane);
@@ -1406,7 +1415,7 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
       return p.cached ? pos - kdiv.q : kdiv.q;
     };
     RotFactor<D> fk_next;
-    load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
+    if (!p.krot) load_factor<D>(fk_next, p, key_anchor(0), lane, interp && sc.remote(0));
     const bool write_cache = p.k_cache_out != nullptr && slot == 0 && p.mode == 0 && !p.cached;
     for (int n = 0; n < sc.n_virt; ++n) {
       const bool remote = sc.remote(n);
@@ -1428,7 +1437,7 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
         if (lane == 0) mbar_arrive(&bars->q_ready);
       }
       const RotFactor<D> fk = fk_next;
-      if (n + 1 < sc.n_virt) load_factor<D>(fk_next, p, key_anchor(n + 1), lane, interp && sc.remote(n + 1));
+      if (n + 1 < sc.n_virt && !p.krot) load_factor<D>(fk_next, p, key_anchor(n + 1), lane, interp && sc.remote(n + 1));
       const int s = n % Lay::kKStages;
       {
         const int first = sc.kt(n) * kBN + RR * rw, last = min(first + RR - 1, L - 1);
@@ -1442,7 +1451,9 @@ __global__ void __launch_bounds__(PrefillDbLayout<D>::kThreads, 1)
       if (!mbar_wait(&bars->k_full[s], (n / Lay::kKStages) & 1, abort)) break;
       if (rw < 4) JL_TRACE_AT(n, 6 + 3 * rw);
       uint8_t* tile = sK + s * Lay::kTileBytes;
-      if (!p.cached) {
+      if (p.krot) {
+        // the keys arrived rotated for this visit's kind
+      } else if (!p.cached) {
         rotate_slice_any<D, RR>(tile, rw, sc.kt(n) * kBN, g, fk, stp, lane);
         if (write_cache && !remote && sc.kt(n) == qt) {
           __syncwarp();

@@ -39,11 +39,12 @@ SIGNATURES = {
     "jl_decode_single_launch_enabled": (ctypes.c_int, []),
     "jl_rope_tables": (ctypes.c_int, [_vp, _vp, _i64, _i32, _f64, _vp]),
     "jl_bifocal_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32,
-                                          _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
+                                          _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "jl_bifocal_prefill_workspace_size": (_sz, [_i64, _i32, _i32]),
     "jl_bifocal_prefill_and_cache": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
                                                     _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _vp, _i64, _vp]),
     "jl_plain_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
-                                        _f32, _vp, _vp, _vp]),
+                                        _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
                                          _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
@@ -189,16 +190,35 @@ def _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse):
     return T, hq, k.shape[1], d, out, lse
 
 
+def jl_bifocal_prefill_workspace_size(total_tokens: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(_lib.jl_bifocal_prefill_workspace_size(total_tokens, n_kv_heads, head_dim))
+
+
+def _key_workspace(workspace, rotate_keys_in_kernel, T, hkv, d, device):
+    """(pointer, bytes) of the prefill's key workspace: the caller's tensor, a new one
+    (workspace=None), or none at all when the kernel is to rotate the keys itself."""
+    if rotate_keys_in_kernel:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(jl_bifocal_prefill_workspace_size(T, hkv, d), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
 def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, *,
-                       softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True, stream=None):
+                       softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True, workspace=None,
+                       rotate_keys_in_kernel: bool = False, stream=None):
     """Bifocal prefill over packed sequences. q [T][Hq][d], k/v [T][Hkv][d] raw bf16.
 
-    Returns (out bf16 [T][Hq][d], lse fp32 [Hq][T] or None)."""
+    The keys are rotated once into a workspace (workspace=None allocates one) unless
+    rotate_keys_in_kernel is set.  Returns (out bf16 [T][Hq][d], lse fp32 [Hq][T] or None)."""
     T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
     batch = cu_seqlens.shape[0] - 1
+    ws, ws_bytes = _key_workspace(workspace, rotate_keys_in_kernel, T, hkv, d, q.device)
     _check(_lib.jl_bifocal_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq, hkv, d,
                                    w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out),
-                                   _ptr(lse), _stream(stream)), "jl_bifocal_prefill")
+                                   _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)), "jl_bifocal_prefill")
     return out, lse
 
 
@@ -263,13 +283,15 @@ def jl_bifocal_prefill_and_cache(q, k, v, cu_seqlens, max_seqlen: int, w0: int, 
 
 
 def jl_plain_prefill(q, k, v, cu_seqlens, max_seqlen: int, cos, sin, *, softmax_scale: float = 0.0, out=None,
-                     lse=None, want_lse: bool = True, stream=None):
-    """Plain causal RoPE prefill (comparator), same layout as jl_bifocal_prefill."""
+                     lse=None, want_lse: bool = True, workspace=None, rotate_keys_in_kernel: bool = False,
+                     stream=None):
+    """Plain causal RoPE prefill (comparator), same layout and key workspace as jl_bifocal_prefill."""
     T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
     batch = cu_seqlens.shape[0] - 1
+    ws, ws_bytes = _key_workspace(workspace, rotate_keys_in_kernel, T, hkv, d, q.device)
     _check(_lib.jl_plain_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq, hkv, d,
                                  _ptr(cos), _ptr(sin), cos.shape[0], softmax_scale, _ptr(out), _ptr(lse),
-                                 _stream(stream)), "jl_plain_prefill")
+                                 _ptr(ws), ws_bytes, _stream(stream)), "jl_plain_prefill")
     return out, lse
 
 

@@ -51,16 +51,18 @@ def test_group_size_matches_golden(jlmod):
 
 def _call_prefill(jlmod, **over):
     a = dict(q=16, k=16, v=16, cu=16, batch=1, T=256, max_seqlen=256, Hq=1, Hkv=1, d=64, w0=32, w_pre=64,
-             cos=16, sin=16, n_tab=256, scale=0.0, out=16, lse=16, stream=None)
+             cos=16, sin=16, n_tab=256, scale=0.0, out=16, lse=16, ws=None, ws_bytes=0, stream=None)
     a.update(over)
     return jlmod._lib.jl_bifocal_prefill(a["q"], a["k"], a["v"], a["cu"], a["batch"], a["T"], a["max_seqlen"],
                                          a["Hq"], a["Hkv"], a["d"], a["w0"], a["w_pre"], a["cos"], a["sin"],
-                                         a["n_tab"], a["scale"], a["out"], a["lse"], a["stream"])
+                                         a["n_tab"], a["scale"], a["out"], a["lse"], a["ws"], a["ws_bytes"],
+                                         a["stream"])
 
 
 @pytest.mark.parametrize("over,status", [
     (dict(d=96), 2), (dict(Hq=3, Hkv=2), 1), (dict(w0=-1), 1), (dict(w_pre=0), 1), (dict(n_tab=100), 1),
     (dict(q=None), 1), (dict(q=24), 1), (dict(batch=-1), 1), (dict(T=-5), 1), (dict(T=1 << 31), 1),
+    (dict(ws=16, ws_bytes=1000), 1), (dict(ws=24, ws_bytes=1 << 20), 1),
 ])
 def test_prefill_rejects_bad_arguments_without_launching(jlmod, over, status):
     # the pointers are fake host addresses: a launch would fail, validation must stop first
@@ -131,3 +133,9 @@ def test_rope_tables_rejects_bad_arguments(jlmod):
 def test_selftest_rejects_bad_limits(jlmod):
     assert jlmod._lib.jl_selftest_wait_timeout(10, None) == 1
     assert jlmod._lib.jl_selftest_wait_timeout(3_000_000_000, None) == 1
+
+
+def test_prefill_workspace_size(jlmod):
+    # two rotated key rows (base and remote) per token and KV head
+    assert jlmod.jl_bifocal_prefill_workspace_size(131072, 8, 128) == 2 * 131072 * 8 * 128 * 2
+    assert jlmod.jl_bifocal_prefill_workspace_size(0, 8, 128) == 0

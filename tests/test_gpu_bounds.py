@@ -2,7 +2,8 @@
 -DJL_DEBUG_BOUNDS (libjetlong_bounds.so) checks, on the device, every index its
 kernels derive there (RoPE table rows, TMA tile coordinates, cache and page
 positions, workspace slots) and records a failed check in the status word
-instead of trapping.  Every product kernel runs here on small parity cases; each
+instead of trapping.  The prefill runs both ways: keys rotated once into a
+workspace (the default), and rotated by the prefill kernel itself.  Every product kernel runs here on small parity cases; each
 must pass its oracle comparison with no check failing.  A paged decode given a
 page index outside its pool (which the normal build reads as zeros) must be
 reported.  This is the stand-in for a memory checker on this machine.
@@ -46,6 +47,14 @@ def test_bounds_build_prefill(jlb, name):
     case = next(c for c in P.SMALL if c[0] == name)
     _, seqlens, hq, hkv, d, w0, w_pre = case
     P._compare_all_rows(jlb, I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True))
+
+
+@pytest.mark.parametrize("name", ["gqa4_G4_w0_100", "varlen_ragged", "group3_d64", "group3_d128_G4"])
+def test_bounds_build_prefill_in_kernel_key_rotation(jlb, name):
+    """The path without a key workspace: the prefill kernel's rotation warps rotate the keys."""
+    case = next(c for c in P.SMALL if c[0] == name)
+    _, seqlens, hq, hkv, d, w0, w_pre = case
+    P._compare_all_rows(jlb, I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True), in_kernel=True)
 
 
 def test_bounds_build_tiny_and_empty_sequences(jlb):

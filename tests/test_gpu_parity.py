@@ -43,14 +43,17 @@ def _check(got_out, got_lse, ref_out, ref_lse, what):
     return err.max(), err.mean(), lerr.max()
 
 
-def _prefill_gpu(jl, q, k, v, cu, cfg, plain=False):
+def _prefill_gpu(jl, q, k, v, cu, cfg, plain=False, in_kernel=False):
+    """in_kernel: the prefill kernel rotates the keys itself (no key workspace); otherwise
+    the keys are rotated once into a workspace before it (the default path)."""
     dev = "cuda"
     qd, kd, vd, cud = q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
     cos, sin = _tables(jl, max(cfg.max_seqlen, 1), cfg.head_dim, cfg.rope_base)
     if plain:
-        out, lse = jl.jl_plain_prefill(qd, kd, vd, cud, cfg.max_seqlen, cos, sin)
+        out, lse = jl.jl_plain_prefill(qd, kd, vd, cud, cfg.max_seqlen, cos, sin, rotate_keys_in_kernel=in_kernel)
     else:
-        out, lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, cfg.w0, cfg.w_pretrained, cos, sin)
+        out, lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, cfg.w0, cfg.w_pretrained, cos, sin,
+                                         rotate_keys_in_kernel=in_kernel)
     jl.jl_sync_status()
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
@@ -62,9 +65,9 @@ def _oracle_rows(q, k, v, cu, cfg, seq, rows, heads, plain=False):
                           rope_base=cfg.rope_base, plain=plain)
 
 
-def _compare_all_rows(jl, cfg, plain=False):
+def _compare_all_rows(jl, cfg, plain=False, in_kernel=False):
     q, k, v, cu = I.prefill_inputs(cfg)
-    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg, plain)
+    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg, plain, in_kernel)
     for s in range(len(cfg.seqlens)):
         L = cfg.seqlens[s]
         if L == 0:
@@ -73,7 +76,8 @@ def _compare_all_rows(jl, cfg, plain=False):
         head = np.tile(np.arange(cfg.n_q_heads), L)
         ro, rl = _oracle_rows(q, k, v, cu, cfg, s, pos, head, plain)
         s0 = int(cu[s])
-        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{cfg.name} seq {s}")
+        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl,
+               f"{cfg.name} seq {s}" + (" (in-kernel key rotation)" if in_kernel else ""))
     return out, lse
 
 
@@ -117,6 +121,12 @@ def test_tiny_plain_prefill_all_rows(jl):
     _compare_all_rows(jl, I.TINY, plain=True)
 
 
+def test_tiny_prefill_in_kernel_key_rotation(jl):
+    """The path without a key workspace: the prefill kernel rotates every key tile itself."""
+    _compare_all_rows(jl, I.TINY, in_kernel=True)
+    _compare_all_rows(jl, I.TINY, plain=True, in_kernel=True)
+
+
 SMALL = [
     # name, seqlens, Hq, Hkv, d, w0, w_pre
     ("gqa4_G4_w0_100", (1000,), 8, 2, 128, 100, 256),
@@ -148,6 +158,34 @@ def test_small_prefill_all_rows(jl, case):
     _compare_all_rows(jl, cfg)
 
 
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_prefill_in_kernel_key_rotation(jl, case):
+    name, seqlens, hq, hkv, d, w0, w_pre = case
+    cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
+    _compare_all_rows(jl, cfg, in_kernel=True)
+
+
+def test_prefill_key_workspace_contents_do_not_matter(jl):
+    """A key workspace full of random bytes and one of zeros give the same result, bit for
+    bit: every row the kernel reads is written by the key rotation first (the remote rows
+    of a G = 1 sequence are neither written nor read)."""
+    cfg = I.PrefillConfig("ws_garbage", (700, 64, 300), 8, 2, 128, 100, 256, 1e4, True)
+    q, k, v, cu = I.prefill_inputs(cfg)
+    dev = "cuda"
+    qd, kd, vd, cud = q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
+    cos, sin = _tables(jl, cfg.max_seqlen, cfg.head_dim, cfg.rope_base)
+    n = jl.jl_bifocal_prefill_workspace_size(qd.shape[0], cfg.n_kv_heads, cfg.head_dim)
+    gen = torch.Generator(device="cpu").manual_seed(3)
+    results = []
+    for ws in (torch.randint(0, 256, (n,), dtype=torch.uint8, generator=gen).to(dev),
+               torch.zeros(n, dtype=torch.uint8, device=dev)):
+        out, lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, cfg.w0, cfg.w_pretrained, cos, sin,
+                                         workspace=ws)
+        jl.jl_sync_status()
+        results.append((out.clone(), lse.clone()))
+    assert torch.equal(results[0][0], results[1][0]) and torch.equal(results[0][1], results[1][1])
+
+
 def test_short_input_gpu_bifocal_equals_plain_bitwise(jl):
     """L <= w_pretrained (G = 1): the kernel takes the plain path, so the outputs are identical."""
     cfg = I.PrefillConfig("G1", (900,), 8, 2, 128, 100, 1024, 1e6, True)
@@ -171,9 +209,9 @@ def _critical_rows(L, w0, w_pre, extra_seed, n_random):
     return sorted(r for r in rows if 0 <= r < L)
 
 
-def _compare_sampled(jl, cfg, n_random=24, heads_per_row=4, seed=11):
+def _compare_sampled(jl, cfg, n_random=24, heads_per_row=4, seed=11, in_kernel=False):
     q, k, v, cu = I.prefill_inputs(cfg)
-    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg)
+    out, lse = _prefill_gpu(jl, q, k, v, cu, cfg, in_kernel=in_kernel)
     rng = np.random.default_rng(seed)
     worst = (0.0, 0.0, 0.0)
     for s in range(len(cfg.seqlens)):
@@ -200,6 +238,10 @@ def test_qwen3_1p7b_64k_sampled_rows(jl, w0):
 
 def test_qwen3_8b_128k_sampled_rows(jl):
     _compare_sampled(jl, I.QWEN3_8B_128K, n_random=24)
+
+
+def test_qwen3_8b_128k_sampled_rows_in_kernel_key_rotation(jl):
+    _compare_sampled(jl, I.QWEN3_8B_128K, n_random=12, in_kernel=True)
 
 
 @pytest.mark.parametrize("L", [32768, 32769])
@@ -507,8 +549,9 @@ PREFILL_AND_CACHE = [
 
 @pytest.mark.parametrize("case", PREFILL_AND_CACHE, ids=[c[0] for c in PREFILL_AND_CACHE])
 def test_prefill_and_cache_writes_the_base_rope_cache(jl, case):
-    """Same attention as jl_bifocal_prefill, bit for bit; the cache holds R(p) k (one bf16
-    rounding of fp32 math) and v for every position of every sequence, nothing beyond."""
+    """Same attention as jl_bifocal_prefill with in-kernel key rotation, bit for bit; the
+    cache holds R(p) k (one bf16 rounding of fp32 math) and v for every position of every
+    sequence, nothing beyond."""
     name, seqlens, hq, hkv, d, w0, w_pre = case
     cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
     q, k, v, cu = I.prefill_inputs(cfg)
@@ -518,7 +561,8 @@ def test_prefill_and_cache_writes_the_base_rope_cache(jl, case):
     cos, sin = _tables(jl, stride, d, cfg.rope_base)
     qd, kd, vd, cud = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
     out, lse = jl.jl_bifocal_prefill_and_cache(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin, kc, vc)
-    ref_out, ref_lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin)
+    ref_out, ref_lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin,
+                                             rotate_keys_in_kernel=True)
     jl.jl_sync_status()
     assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
     kc, vc = kc.cpu(), vc.cpu()
