@@ -193,17 +193,23 @@ size_t jl_bifocal_prefill_workspace_size(int64_t total_tokens, int32_t Hkv, int3
  *   k_cache, v_cache  bf16 [batch][cache_stride][Hkv][head_dim], caller-owned,
  *                     16-byte aligned; positions >= the sequence length are not written
  *   cache_stride      >= max_seqlen
- * The kernel writes each key tile while it holds it rotated for its own query
- * block (one CTA per KV head and block), so the cache costs no extra pass over K.
- * w0 = 0 has no base-position visit when G > 1; then the cache is written by
- * the cache-writer kernel (jl_kv_cache_fill) after the attention.
+ *   workspace, workspace_bytes  as for jl_bifocal_prefill.  With a workspace the
+ *                     keys are rotated once into it, the attention is exactly
+ *                     jl_bifocal_prefill's with a workspace, and the cache writer
+ *                     (jl_kv_cache_fill) fills the cache.  Without one (NULL, 0)
+ *                     the kernel rotates the keys itself and writes each key tile
+ *                     while it holds it rotated for its own query block (one CTA
+ *                     per KV head and block), so the cache costs no extra pass
+ *                     over K; w0 = 0 has no base-position visit when G > 1, and
+ *                     then the cache writer fills the cache after the attention.
  */
 jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
                                        int32_t batch, int64_t total_tokens, int32_t max_seqlen, int32_t Hq,
                                        int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
                                        const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
                                        float softmax_scale, void* out, float* lse, void* k_cache, void* v_cache,
-                                       int64_t cache_stride, jl_stream_t stream);
+                                       int64_t cache_stride, void* workspace, size_t workspace_bytes,
+                                       jl_stream_t stream);
 
 /*
  * Chunked prefill against a base-RoPE cache (a prompt processed in pieces, or

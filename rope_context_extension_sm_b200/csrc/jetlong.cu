@@ -707,11 +707,24 @@ jl_status jl_bifocal_prefill_and_cache(const void* q, const void* k, const void*
                                        int32_t Hkv, int32_t head_dim, int32_t w0, int32_t w_pretrained,
                                        const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
                                        float softmax_scale, void* out, float* lse, void* k_cache, void* v_cache,
-                                       int64_t cache_stride, jl_stream_t stream) {
+                                       int64_t cache_stride, void* workspace, size_t workspace_bytes,
+                                       jl_stream_t stream) {
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cache_stride < max_seqlen || cache_stride < 1)
     return fail(JL_ERR_INVALID, "cache_stride (%lld) must be >= max_seqlen (%d) and >= 1", (long long)cache_stride,
                 max_seqlen);
+  if (workspace != nullptr) {
+    // Keys rotated once into the workspace: the attention is jl_bifocal_prefill's with
+    // that workspace, and the cache writer fills the cache beside it.
+    if (batch > 0 && total_tokens > 0 && max_seqlen > 0 && (!k_cache || !v_cache))
+      return fail(JL_ERR_INVALID, "null cache pointer");
+    jl_status s = prefill_common(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
+                                 w_pretrained, 0, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, workspace,
+                                 workspace_bytes, st);
+    if (s != JL_OK || batch == 0 || total_tokens == 0 || max_seqlen == 0) return s;
+    return append_common(nullptr, k, v, cu_seqlens, nullptr, batch, total_tokens, 0, Hkv, head_dim, cos_tab,
+                         sin_tab, n_tab_rows, nullptr, k_cache, v_cache, cache_stride, nullptr, 0, 0, 0, st, true);
+  }
   jl::PrefillParams prm;
   bool empty;
   jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,

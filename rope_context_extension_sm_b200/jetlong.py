@@ -42,7 +42,8 @@ SIGNATURES = {
                                           _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_prefill_workspace_size": (_sz, [_i64, _i32, _i32]),
     "jl_bifocal_prefill_and_cache": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32,
-                                                    _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _vp, _i64, _vp]),
+                                                    _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _vp, _i64, _vp, _sz,
+                                                    _vp]),
     "jl_plain_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
                                         _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _i32, _vp,
@@ -266,19 +267,22 @@ def jl_bifocal_prefill_three_pass(q, k, v, cu_seqlens, max_seqlen: int, w0: int,
 
 def jl_bifocal_prefill_and_cache(q, k, v, cu_seqlens, max_seqlen: int, w0: int, w_pretrained: int, cos, sin, k_cache,
                                  v_cache, *, softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True,
-                                 stream=None):
+                                 workspace=None, rotate_keys_in_kernel: bool = False, stream=None):
     """jl_bifocal_prefill that also writes the base-RoPE cache: k_cache[b][j] = R(j) k_j,
-    v_cache[b][j] = v_j, caches [batch][stride][Hkv][d] bf16.  Returns (out, lse)."""
+    v_cache[b][j] = v_j, caches [batch][stride][Hkv][d] bf16.  Key workspace as for
+    jl_bifocal_prefill.  Returns (out, lse)."""
     T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
     _need(k_cache, torch.bfloat16, "k_cache", 4)
     _need(v_cache, torch.bfloat16, "v_cache", 4)
     if k_cache.shape != v_cache.shape or k_cache.shape[2:] != (hkv, d):
         raise ValueError("k_cache and v_cache must both be [batch][stride][Hkv][d]")
     batch = cu_seqlens.shape[0] - 1
+    ws, ws_bytes = _key_workspace(workspace, rotate_keys_in_kernel, T, hkv, d, q.device)
     _check(_lib.jl_bifocal_prefill_and_cache(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq,
                                              hkv, d, w0, w_pretrained, _ptr(cos), _ptr(sin), cos.shape[0],
                                              softmax_scale, _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache),
-                                             k_cache.shape[1], _stream(stream)), "jl_bifocal_prefill_and_cache")
+                                             k_cache.shape[1], _ptr(ws), ws_bytes, _stream(stream)),
+           "jl_bifocal_prefill_and_cache")
     return out, lse
 
 

@@ -116,11 +116,13 @@ def test_prefill_and_cache_rejects_a_short_cache_without_launching(jlmod):
     lib = jlmod._lib
     # cache_stride below max_seqlen is refused before any pointer is touched or kernel launched
     st = lib.jl_bifocal_prefill_and_cache(None, None, None, None, 1, 100, 100, 4, 2, 128, 16, 64, None, None, 128,
-                                          0.0, None, None, None, None, 99, None)
+                                          0.0, None, None, None, None, 99, None, 0, None)
     assert st == 1 and "cache_stride" in jlmod.jl_last_error()
     # an empty batch is a no-op, whatever the pointers
     assert lib.jl_bifocal_prefill_and_cache(None, None, None, None, 0, 0, 0, 4, 2, 128, 16, 64, None, None, 1,
-                                            0.0, None, None, None, None, 1, None) == 0
+                                            0.0, None, None, None, None, 1, None, 0, None) == 0
+    assert lib.jl_bifocal_prefill_and_cache(None, None, None, None, 0, 0, 0, 4, 2, 128, 16, 64, None, None, 1,
+                                            0.0, None, None, None, None, 1, 16, 1 << 20, None) == 0
 
 
 def test_rope_tables_rejects_bad_arguments(jlmod):

@@ -62,9 +62,10 @@ def test_bounds_build_tiny_and_empty_sequences(jlb):
     P._compare_all_rows(jlb, I.PrefillConfig("with_empty", (0, 200, 0, 5), 2, 1, 128, 16, 64, 1e4, False))
 
 
+@pytest.mark.parametrize("in_kernel", [False, True], ids=["key_workspace", "in_kernel_rotation"])
 @pytest.mark.parametrize("case", P.PREFILL_AND_CACHE, ids=[c[0] for c in P.PREFILL_AND_CACHE])
-def test_bounds_build_prefill_and_cache(jlb, case):
-    P.test_prefill_and_cache_writes_the_base_rope_cache(jlb, case)
+def test_bounds_build_prefill_and_cache(jlb, case, in_kernel):
+    P.test_prefill_and_cache_writes_the_base_rope_cache(jlb, case, in_kernel)
 
 
 def test_bounds_build_chunked_three_pass_interp(jlb):

@@ -547,10 +547,11 @@ PREFILL_AND_CACHE = [
 ]
 
 
+@pytest.mark.parametrize("in_kernel", [False, True], ids=["key_workspace", "in_kernel_rotation"])
 @pytest.mark.parametrize("case", PREFILL_AND_CACHE, ids=[c[0] for c in PREFILL_AND_CACHE])
-def test_prefill_and_cache_writes_the_base_rope_cache(jl, case):
-    """Same attention as jl_bifocal_prefill with in-kernel key rotation, bit for bit; the
-    cache holds R(p) k (one bf16 rounding of fp32 math) and v for every position of every
+def test_prefill_and_cache_writes_the_base_rope_cache(jl, case, in_kernel):
+    """Same attention as jl_bifocal_prefill on the same key path, bit for bit; the cache
+    holds R(p) k (one bf16 rounding of fp32 math) and v for every position of every
     sequence, nothing beyond."""
     name, seqlens, hq, hkv, d, w0, w_pre = case
     cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, w_pre, 1e4, True)
@@ -560,9 +561,10 @@ def test_prefill_and_cache_writes_the_base_rope_cache(jl, case):
     vc = torch.zeros_like(kc)
     cos, sin = _tables(jl, stride, d, cfg.rope_base)
     qd, kd, vd, cud = q.cuda(), k.cuda(), v.cuda(), cu.cuda()
-    out, lse = jl.jl_bifocal_prefill_and_cache(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin, kc, vc)
+    out, lse = jl.jl_bifocal_prefill_and_cache(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin, kc, vc,
+                                               rotate_keys_in_kernel=in_kernel)
     ref_out, ref_lse = jl.jl_bifocal_prefill(qd, kd, vd, cud, cfg.max_seqlen, w0, w_pre, cos, sin,
-                                             rotate_keys_in_kernel=True)
+                                             rotate_keys_in_kernel=in_kernel)
     jl.jl_sync_status()
     assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
     kc, vc = kc.cpu(), vc.cpu()
