@@ -132,14 +132,16 @@ jl_status jl_rope_tables_scaled(float* cos_out, float* sin_out, int64_t n_pos, i
  * (0 <= i-j < w0) keep base RoPE from cos_tab/sin_tab; every other causal pair
  * scores <R'(i) q, R'(j) k> with R' read from cos_rem/sin_rem at the raw
  * positions (from jl_rope_tables_scaled).  No G or f: the caller's table sets
- * the compression.  Same layout, conventions and kernel as jl_bifocal_prefill;
- * n_rem_rows >= max_seqlen.
+ * the compression.  Same layout, conventions, key workspace (its remote rows are
+ * the interpolated rotation at the raw position) and kernel as
+ * jl_bifocal_prefill; n_rem_rows >= max_seqlen.
  */
 jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
                             int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                             int32_t w0, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
                             const float* cos_rem, const float* sin_rem, int64_t n_rem_rows, float softmax_scale,
-                            void* out, float* lse, jl_stream_t stream);
+                            void* out, float* lse, void* workspace, size_t workspace_bytes,
+                            jl_stream_t stream);
 
 /*
  * Bifocal prefill (Methodology section 2, inclusion-exclusion attention merge).

@@ -268,21 +268,13 @@ size_t key_rot_bytes(int64_t total_tokens, int32_t Hkv, int32_t head_dim) {
   return 2 * static_cast<size_t>(total_tokens) * Hkv * head_dim * sizeof(__nv_bfloat16);
 }
 
-// With a workspace, the keys are rotated once into it (jl_key_rotate_kernel) and the
-// prefill kernel reads them as they are; without one, its rotation warps rotate every
-// key tile on every visit.
-jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
-                         int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
-                         int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
-                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
-                         size_t workspace_bytes, cudaStream_t st) {
-  jl::PrefillParams prm;
-  bool empty;
-  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
-                               w_pretrained, plain, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
-                               &empty);
-  if (s != JL_OK || empty) return s;
-  if (workspace == nullptr) return launch_prefill_any(q, k, v, prm, head_dim, st);
+// Rotates the prompt keys once into the workspace (jl_key_rotate_kernel): base rows
+// R(j) k, then remote rows R(f(j)) k (w_pre gives G per sequence), or with cos_rem the
+// interpolated rotation at the raw position.
+jl_status rotate_keys(const void* k, const int32_t* cu_seqlens, int32_t batch, int64_t total_tokens, int32_t Hkv,
+                      int32_t head_dim, int32_t w_pre, const float* cos_tab, const float* sin_tab,
+                      int64_t n_tab_rows, const float* cos_rem, const float* sin_rem, int64_t n_rem_rows,
+                      void* workspace, size_t workspace_bytes, cudaStream_t st) {
   const size_t need = key_rot_bytes(total_tokens, Hkv, head_dim);
   if (workspace_bytes < need)
     return fail(JL_ERR_INVALID, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
@@ -299,13 +291,38 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
   ap.n_tab_rows = n_tab_rows;
   ap.batch = batch;
   ap.Hkv = Hkv;
-  ap.w_pre = plain ? 0x7fffffff : w_pretrained;  // plain: every pair is local, no remote rows
+  ap.w_pre = w_pre;
+  ap.cos_rem = cos_rem;
+  ap.sin_rem = sin_rem;
+  ap.n_rem_rows = n_rem_rows;
   const int64_t warps = (total_tokens * Hkv + jl::kFillRowsPerWarp - 1) / jl::kFillRowsPerWarp;
   const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
   if (head_dim == 128) jl::jl_key_rotate_kernel<128><<<blocks, 256, 0, st>>>(ap);
   else jl::jl_key_rotate_kernel<64><<<blocks, 256, 0, st>>>(ap);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "key rotation launch");
+  return ok();
+}
+
+// With a workspace, the keys are rotated once into it (jl_key_rotate_kernel) and the
+// prefill kernel reads them as they are; without one, its rotation warps rotate every
+// key tile on every visit.
+jl_status prefill_common(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int32_t batch,
+                         int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                         int32_t w0, int32_t w_pretrained, int plain, const float* cos_tab, const float* sin_tab,
+                         int64_t n_tab_rows, float softmax_scale, void* out, float* lse, void* workspace,
+                         size_t workspace_bytes, cudaStream_t st) {
+  jl::PrefillParams prm;
+  bool empty;
+  jl_status s = prefill_params(q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, Hq, Hkv, head_dim, w0,
+                               w_pretrained, plain, cos_tab, sin_tab, n_tab_rows, softmax_scale, out, lse, &prm,
+                               &empty);
+  if (s != JL_OK || empty) return s;
+  if (workspace == nullptr) return launch_prefill_any(q, k, v, prm, head_dim, st);
+  // plain: every pair is local, so no remote rows
+  if ((s = rotate_keys(k, cu_seqlens, batch, total_tokens, Hkv, head_dim, plain ? 0x7fffffff : w_pretrained,
+                       cos_tab, sin_tab, n_tab_rows, nullptr, nullptr, 0, workspace, workspace_bytes, st)) != JL_OK)
+    return s;
   prm.krot = 1;
   return launch_prefill_any(q, workspace, v, prm, head_dim, st);
 }
@@ -653,7 +670,7 @@ jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const i
                             int64_t total_tokens, int32_t max_seqlen, int32_t Hq, int32_t Hkv, int32_t head_dim,
                             int32_t w0, const float* cos_tab, const float* sin_tab, int64_t n_tab_rows,
                             const float* cos_rem, const float* sin_rem, int64_t n_rem_rows, float softmax_scale,
-                            void* out, float* lse, jl_stream_t stream) {
+                            void* out, float* lse, void* workspace, size_t workspace_bytes, jl_stream_t stream) {
   if (!cos_rem || !sin_rem) return fail(JL_ERR_INVALID, "null remote table");
   if (n_rem_rows < max_seqlen)
     return fail(JL_ERR_INVALID, "n_rem_rows (%lld) must be >= max_seqlen (%d)", (long long)n_rem_rows, max_seqlen);
@@ -666,7 +683,14 @@ jl_status jl_interp_prefill(const void* q, const void* k, const void* v, const i
   prm.cos_rem = cos_rem;
   prm.sin_rem = sin_rem;
   prm.n_rem_rows = n_rem_rows;
-  return launch_prefill_any(q, k, v, prm, head_dim, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (workspace == nullptr) return launch_prefill_any(q, k, v, prm, head_dim, st);
+  // remote rows: the interpolated rotation at the raw position, for every sequence
+  if ((s = rotate_keys(k, cu_seqlens, batch, total_tokens, Hkv, head_dim, 1, cos_tab, sin_tab, n_tab_rows, cos_rem,
+                       sin_rem, n_rem_rows, workspace, workspace_bytes, st)) != JL_OK)
+    return s;
+  prm.krot = 1;
+  return launch_prefill_any(q, workspace, v, prm, head_dim, st);
 }
 
 jl_status jl_rope_tables(float* cos_out, float* sin_out, int64_t n_pos, int32_t head_dim, double rope_base,

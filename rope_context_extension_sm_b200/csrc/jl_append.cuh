@@ -37,6 +37,9 @@ struct AppendParams {
   const int32_t* block_table;  // paged caches (NULL: contiguous [batch][cache_stride])
   int32_t page_size, max_pages, num_pages;
   int32_t w_pre;               // key rotation: w_pretrained, for G per sequence
+  const float* cos_rem;        // key rotation, interpolation variant: remote rows rotate by
+  const float* sin_rem;        // these tables at raw positions (NULL: R(f(j)))
+  int64_t n_rem_rows;
 };
 
 // Cache row of entry b's position pos (already checked against cache_stride):
@@ -167,6 +170,8 @@ __global__ void __launch_bounds__(256) jl_kv_fill_kernel(const AppendParams p) {
 //   k_out[t]     = R(j) k_t          (local visits)
 //   k_out[T + t] = R(floor(j / G)) k_t  (remote visits; not written for G = 1, whose
 //                                       pairs are all local)
+// For the interpolation variant (p.cos_rem set) the remote rows are rotated by the
+// interpolated tables at the raw position j, for every sequence.
 // Same lane layout and load batching as jl_kv_fill_kernel; p.k_cache is the output.
 template <int D>
 __global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p) {
@@ -176,6 +181,8 @@ __global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p
   const int lane = threadIdx.x & 31;
   const int64_t n_rows = p.total_tokens * p.Hkv;
   const int64_t remote_off = p.total_tokens * p.Hkv * D;  // element offset of the remote rows
+  const float* rcos = p.cos_rem != nullptr ? p.cos_rem : p.cos_tab;  // tables of the remote rows
+  const float* rsin = p.sin_rem != nullptr ? p.sin_rem : p.sin_tab;
   int64_t src[R], pos[R], fpos[R];
   bool live[R];
 #pragma unroll
@@ -201,7 +208,16 @@ __global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p
       live[r] = false;
       continue;
     }
-    if (G > 1) fpos[r] = pos[r] / G;
+    if (p.cos_rem != nullptr) {
+      if (pos[r] >= p.n_rem_rows) {  // the host checks max_seqlen <= n_rem_rows
+        if (lane == 0) atomicOr(&g_status, kDevErrBounds);
+        live[r] = false;
+        continue;
+      }
+      fpos[r] = pos[r];
+    } else if (G > 1) {
+      fpos[r] = pos[r] / G;
+    }
     src[r] = (t * p.Hkv + h) * D;
   }
   if constexpr (D == 128) {
@@ -215,8 +231,8 @@ __global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p
       cs[r] = *reinterpret_cast<const float2*>(p.cos_tab + pos[r] * HALF + 2 * lane);
       sn[r] = *reinterpret_cast<const float2*>(p.sin_tab + pos[r] * HALF + 2 * lane);
       const int64_t fr = fpos[r] >= 0 ? fpos[r] : 0;
-      cf[r] = *reinterpret_cast<const float2*>(p.cos_tab + fr * HALF + 2 * lane);
-      sf[r] = *reinterpret_cast<const float2*>(p.sin_tab + fr * HALF + 2 * lane);
+      cf[r] = *reinterpret_cast<const float2*>(rcos + fr * HALF + 2 * lane);
+      sf[r] = *reinterpret_cast<const float2*>(rsin + fr * HALF + 2 * lane);
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -243,8 +259,8 @@ __global__ void __launch_bounds__(256) jl_key_rotate_kernel(const AppendParams p
       cs[r] = p.cos_tab[pos[r] * HALF + lane];
       sn[r] = p.sin_tab[pos[r] * HALF + lane];
       const int64_t fr = fpos[r] >= 0 ? fpos[r] : 0;
-      cf[r] = p.cos_tab[fr * HALF + lane];
-      sf[r] = p.sin_tab[fr * HALF + lane];
+      cf[r] = rcos[fr * HALF + lane];
+      sf[r] = rsin[fr * HALF + lane];
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {

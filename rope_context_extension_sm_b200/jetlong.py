@@ -57,7 +57,7 @@ SIGNATURES = {
     "jl_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
     "jl_rope_tables_scaled": (ctypes.c_int, [_vp, _vp, _i64, _i32, _f64, _vp, _vp]),
     "jl_interp_prefill": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
-                                         _vp, _vp, _i64, _f32, _vp, _vp, _vp]),
+                                         _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_bifocal_decode_paged": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                                _i32, _i32, _i32, _vp, _vp, _i64, _f32, _vp, _vp, _vp, _sz, _vp]),
     "jl_kv_cache_fill_paged": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _i64, _vp, _vp,
@@ -159,15 +159,19 @@ def jl_rope_tables_scaled(n_pos: int, head_dim: int, rope_base: float, freq_scal
 
 
 def jl_interp_prefill(q, k, v, cu_seqlens, max_seqlen: int, w0: int, cos, sin, cos_rem, sin_rem, *,
-                      softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True, stream=None):
-    """Frequency-interpolation variant of the remote window (local pairs base RoPE)."""
+                      softmax_scale: float = 0.0, out=None, lse=None, want_lse: bool = True, workspace=None,
+                      rotate_keys_in_kernel: bool = False, stream=None):
+    """Frequency-interpolation variant of the remote window (local pairs base RoPE).
+    Key workspace as for jl_bifocal_prefill."""
     T, hq, hkv, d, out, lse = _prefill_args(q, k, v, cu_seqlens, cos, sin, out, lse, want_lse)
     _need(cos_rem, torch.float32, "cos_rem", 2)
     _need(sin_rem, torch.float32, "sin_rem", 2)
     batch = cu_seqlens.shape[0] - 1
+    ws, ws_bytes = _key_workspace(workspace, rotate_keys_in_kernel, T, hkv, d, q.device)
     _check(_lib.jl_interp_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, T, max_seqlen, hq, hkv, d, w0,
                                   _ptr(cos), _ptr(sin), cos.shape[0], _ptr(cos_rem), _ptr(sin_rem), cos_rem.shape[0],
-                                  softmax_scale, _ptr(out), _ptr(lse), _stream(stream)), "jl_interp_prefill")
+                                  softmax_scale, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
+           "jl_interp_prefill")
     return out, lse
 
 

@@ -73,7 +73,8 @@ def test_bounds_build_chunked_three_pass_interp(jlb):
     P.test_chunked_prefill_d64_group3(jlb)
     P.test_chunked_prefill_d128_group3(jlb)
     P.test_three_pass_merge_on_gpu(jlb, P.THREE_PASS[0])
-    P.test_interp_prefill_matches_oracle(jlb, P.INTERP[1])
+    P.test_interp_prefill_matches_oracle(jlb, P.INTERP[1], False)
+    P.test_interp_prefill_matches_oracle(jlb, P.INTERP[1], True)
 
 
 @pytest.mark.parametrize("case", [c for c in P.DECODE_GROUPS if c[0] in ("d64_g3", "d64_g16", "d128_g3")],

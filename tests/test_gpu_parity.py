@@ -826,8 +826,11 @@ INTERP = [
 ]
 
 
+@pytest.mark.parametrize("in_kernel", [False, True], ids=["key_workspace", "in_kernel_rotation"])
 @pytest.mark.parametrize("case", INTERP, ids=[c[0] for c in INTERP])
-def test_interp_prefill_matches_oracle(jl, case):
+def test_interp_prefill_matches_oracle(jl, case, in_kernel):
+    """Keys rotated once into a workspace (remote rows: the interpolated rotation at the raw
+    position), or rotated by the prefill kernel itself."""
     name, seqlens, hq, hkv, d, w0, kind, s = case
     cfg = I.PrefillConfig(name, seqlens, hq, hkv, d, w0, 256, 1e4, True)
     lam = np.full(d // 2, 1.0 / s) if kind == "pi" else _yarn_ramp(d, s, cfg.rope_base, 256)
@@ -835,7 +838,8 @@ def test_interp_prefill_matches_oracle(jl, case):
     n = max(cfg.max_seqlen, 1)
     cos, sin = _tables(jl, n, d, cfg.rope_base)
     cr, sr = jl.jl_rope_tables_scaled(n, d, cfg.rope_base, lam)
-    out, lse = jl.jl_interp_prefill(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), cfg.max_seqlen, w0, cos, sin, cr, sr)
+    out, lse = jl.jl_interp_prefill(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), cfg.max_seqlen, w0, cos, sin, cr, sr,
+                                    rotate_keys_in_kernel=in_kernel)
     jl.jl_sync_status()
     out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
     for b, L in enumerate(seqlens):
@@ -844,4 +848,5 @@ def test_interp_prefill_matches_oracle(jl, case):
         head = np.tile(np.arange(hq), L)
         ro, rl = O.interp_rows(I.bf16_bits(q[s0:s0 + L]), I.bf16_bits(k[s0:s0 + L]), I.bf16_bits(v[s0:s0 + L]), L,
                                pos, head, w0=w0, rope_base=cfg.rope_base, freq_scale=lam)
-        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl, f"{name} seq {b}")
+        _check(out[s0 + pos, head], lse[head, s0 + pos], ro, rl,
+               f"{name} seq {b}" + (" (in-kernel key rotation)" if in_kernel else ""))
