@@ -141,3 +141,20 @@ def test_prefill_workspace_size(jlmod):
     # two rotated key rows (base and remote) per token and KV head
     assert jlmod.jl_bifocal_prefill_workspace_size(131072, 8, 128) == 2 * 131072 * 8 * 128 * 2
     assert jlmod.jl_bifocal_prefill_workspace_size(0, 8, 128) == 0
+
+
+def test_key_workspace_is_checked_before_any_launch(jlmod):
+    """A key workspace too small or not 16-byte aligned is refused by every prefill entry
+    point that takes one, before anything is launched (the pointers are fake host addresses)."""
+    lib = jlmod._lib
+    T, hkv, d = 256, 1, 64
+    need = jlmod.jl_bifocal_prefill_workspace_size(T, hkv, d)
+    for ws, nbytes in ((16, need - 16), (24, need)):
+        st = lib.jl_bifocal_prefill_and_cache(16, 16, 16, 16, 1, T, T, 1, hkv, d, 32, 64, 16, 16, 256, 0.0, 16, 16,
+                                              16, 16, 256, ws, nbytes, None)
+        assert st == jlmod.JL_ERR_INVALID and "workspace" in jlmod.jl_last_error()
+        st = lib.jl_interp_prefill(16, 16, 16, 16, 1, T, T, 1, hkv, d, 32, 16, 16, 256, 16, 16, 256, 0.0, 16, 16,
+                                   ws, nbytes, None)
+        assert st == jlmod.JL_ERR_INVALID and "workspace" in jlmod.jl_last_error()
+        st = lib.jl_plain_prefill(16, 16, 16, 16, 1, T, T, 1, hkv, d, 16, 16, 256, 0.0, 16, 16, ws, nbytes, None)
+        assert st == jlmod.JL_ERR_INVALID and "workspace" in jlmod.jl_last_error()
