@@ -6,7 +6,9 @@ query / 8 KV heads, head_dim 128, w_pretrained 32768 -> G = 4, w0 = 4096) plus
 one bifocal decode token against a 131072-token base-RoPE cache (Qwen3-4B
 shape: 32 / 8 heads, head_dim 128).  Inputs are seeded synthetic bf16 data
 (rope_context_extension_sm_b200.inputs), resident in HBM before timing; both
-the prefill inputs (1.5 GB) and the cache (512 MiB) are larger than L2.
+the prefill inputs (1.5 GB) and the cache (512 MiB) are larger than L2.  The
+prefill is the whole jl_bifocal_prefill call with a preallocated key workspace:
+the keys' rotation, then the attention kernel.
 
 Prints ONE JSON line (rank 0).  ``value`` is useful prefill TFLOP/s (each causal
 (q, k) pair counted once at 4 * head_dim flops per query head), aggregated over
@@ -304,7 +306,7 @@ def _measure_next_rows(jl, dev, stream, q, k, v, cu, cos, sin, out, lse, fused_m
                              "gbs": round(fill_bytes / (ms * 1e-3) / 1e9, 1),
                              "frac_of_hbm_measured": round(fill_bytes / (ms * 1e-3) / 1e9 / hbm, 4)}
 
-    # the same cache written by the prefill kernel itself, alongside the attention
+    # the same cache written by jl_bifocal_prefill_and_cache alongside the attention (key workspace)
     pac = lambda: jl.jl_bifocal_prefill_and_cache(q, k, v, cu, L, PREFILL.w0, PREFILL.w_pretrained, cos, sin, kc, vc,
                                                   out=out, lse=lse)
     pac()
