@@ -319,8 +319,9 @@ jl_status prefill_common(const void* q, const void* k, const void* v, const int3
                                &empty);
   if (s != JL_OK || empty) return s;
   if (workspace == nullptr) return launch_prefill_any(q, k, v, prm, head_dim, st);
-  // plain: every pair is local, so no remote rows
-  if ((s = rotate_keys(k, cu_seqlens, batch, total_tokens, Hkv, head_dim, plain ? 0x7fffffff : w_pretrained,
+  // plain: every pair is local, so no remote rows (G = 1 for every length below 2^30,
+  // which rotate_keys requires, without overflowing L + w_pre - 1 in int32)
+  if ((s = rotate_keys(k, cu_seqlens, batch, total_tokens, Hkv, head_dim, plain ? (1 << 30) : w_pretrained,
                        cos_tab, sin_tab, n_tab_rows, nullptr, nullptr, 0, workspace, workspace_bytes, st)) != JL_OK)
     return s;
   prm.krot = 1;
